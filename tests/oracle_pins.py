@@ -1,0 +1,372 @@
+"""Pins for the fp64 oracle: facts fixed by the pages and by the mathematics.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with a closed form, an invariant or an independent brute
+force.  ``test_oracle_pins.py`` runs them on the real oracle and
+``test_oracle_mutants.py`` checks that every planted mistake fails at least one.
+
+Passages (page title, section):
+  [cache]   "Transformer : comprendre l'entrainement et l'inference", "Un cache KV simple"
+            (scale 1/sqrt(d), tril(diagonal=past_len) mask, -inf fill, softmax, @ v)
+  [decode]  same page, "Pre-remplissage et decodage"; and
+            "Transformerを実装して少し理解した気になる会(その4)", "KV Cache"
+            (decode = the last query row against every cached key)
+  [xf]      "Come costruire Transformer efficienti in memoria con xFormers ...":
+            causal lower-triangular mask, block-diagonal packed sequences, GQA, ALiBi
+  [flash]   "FlashAttention (2022)", "Il trucco della softmax ...": softmax weights
+            of a row sum to one; the result is exact.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from oracle import BIAS_BLOCKDIAG, BIAS_BLOCKDIAG_CAUSAL, BIAS_CAUSAL, BIAS_NONE
+
+TOL = 1e-12
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol=TOL, what=""):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    with np.errstate(invalid="ignore"):
+        err = np.where(both_inf, 0.0, np.abs(a - b))
+    bad = ~(err <= tol * (1.0 + np.abs(np.where(both_inf, 0.0, b))))
+    assert not bad.any(), f"{what}: max err {np.nanmax(err)}"
+
+
+def _offsets(lens):
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+
+# ---------------------------------------------------------------------------
+# [flash] weights of a row sum to one: v == 1 gives out == 1 for every row that
+# sees at least one key, under every bias kind, GQA and ALiBi.
+# ---------------------------------------------------------------------------
+def pin_weights_sum_to_one(orc):
+    r = _rng(1)
+    B, M, N, Hq, Hkv, D = 2, 7, 9, 4, 2, 8
+    q, k = r.standard_normal((B, M, Hq, D)), r.standard_normal((B, N, Hkv, D))
+    v = np.ones((B, N, Hkv, D))
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        for alibi in (False, True):
+            out, lse = orc.attention(q, k, v, bias=bias, alibi=alibi)
+            _close(out, np.ones_like(out), what=f"sum-to-one bias={bias} alibi={alibi}")
+            assert np.isfinite(lse).all()
+    lens_q, lens_k = [3, 1, 5], [4, 2, 6]
+    sq, sk = _offsets(lens_q), _offsets(lens_k)
+    q1 = r.standard_normal((1, sum(lens_q), Hq, D))
+    k1, v1 = r.standard_normal((1, sum(lens_k), Hkv, D)), np.ones((1, sum(lens_k), Hkv, D))
+    for bias in (BIAS_BLOCKDIAG, BIAS_BLOCKDIAG_CAUSAL):
+        out, _ = orc.attention(q1, k1, v1, bias=bias, seqstart_q=sq, seqstart_k=sk, alibi=True)
+        _close(out, np.ones_like(out), what=f"sum-to-one varlen bias={bias}")
+
+
+# ---------------------------------------------------------------------------
+# [cache] causal, M == N: row 0 sees only key 0, so out_0 = v_0 and
+# lse_0 = scale <q_0, k_0>.
+# ---------------------------------------------------------------------------
+def pin_causal_row0_is_v0(orc):
+    r = _rng(2)
+    B, M, H, D = 2, 6, 3, 8
+    q, k, v = (r.standard_normal((B, M, H, D)) for _ in range(3))
+    scale = 0.37
+    out, lse = orc.attention(q, k, v, bias=BIAS_CAUSAL, scale=scale)
+    _close(out[:, 0], v[:, 0], what="causal row 0 == v0")
+    _close(lse[:, :, 0], scale * np.einsum("bhd,bhd->bh", q[:, 0], k[:, 0]), what="lse row 0")
+
+
+# ---------------------------------------------------------------------------
+# scale = 0 makes every visible score equal, so the output is the plain mean of
+# the visible values and lse = ln(#visible).  This pins the mask (which keys
+# are visible, bottom-right alignment for M != N, [cache]) and the value rows.
+# ---------------------------------------------------------------------------
+def pin_scale_zero_means(orc):
+    r = _rng(3)
+    D, H = 4, 2
+    for (M, N) in ((5, 5), (3, 7), (7, 4)):
+        q = r.standard_normal((1, M, H, D))
+        k, v = r.standard_normal((1, N, H, D)), r.standard_normal((1, N, H, D))
+        out, lse = orc.attention(q, k, v, bias=BIAS_NONE, scale=0.0)
+        _close(out[0], np.broadcast_to(v[0].mean(0), (M, H, D)), what="mean all")
+        _close(lse, np.full((1, H, M), math.log(N)), what="ln N")
+        out, lse = orc.attention(q, k, v, bias=BIAS_CAUSAL, scale=0.0)
+        for i in range(M):
+            n_vis = i + (N - M) + 1  # keys 0 .. i + N - M
+            if n_vis <= 0:
+                _close(out[0, i], np.zeros((H, D)), what="no key -> 0")
+                assert np.all(np.isneginf(lse[0, :, i])), "no key -> lse -inf"
+            else:
+                _close(out[0, i], v[0, :n_vis].mean(0), what=f"causal mean M={M} N={N} i={i}")
+                _close(lse[0, :, i], np.full(H, math.log(n_vis)), what="causal ln count")
+    # packed sequences: means over each row's own sequence
+    lens_q, lens_k = [2, 4, 3], [3, 4, 1]
+    sq, sk = _offsets(lens_q), _offsets(lens_k)
+    q = r.standard_normal((1, 9, H, D))
+    k, v = r.standard_normal((1, 8, H, D)), r.standard_normal((1, 8, H, D))
+    out, lse = orc.attention(q, k, v, bias=BIAS_BLOCKDIAG, scale=0.0, seqstart_q=sq, seqstart_k=sk)
+    outc, lsec = orc.attention(q, k, v, bias=BIAS_BLOCKDIAG_CAUSAL, scale=0.0, seqstart_q=sq,
+                               seqstart_k=sk)
+    for s in range(3):
+        vs = v[0, sk[s]:sk[s + 1]]
+        m_s, n_s = lens_q[s], lens_k[s]
+        for il in range(m_s):
+            i = sq[s] + il
+            _close(out[0, i], vs.mean(0), what="blockdiag mean")
+            _close(lse[0, :, i], np.full(H, math.log(n_s)), what="blockdiag ln")
+            n_vis = il + (n_s - m_s) + 1
+            if n_vis <= 0:
+                assert np.all(np.isneginf(lsec[0, :, i]))
+                _close(outc[0, i], np.zeros((H, D)))
+            else:
+                _close(outc[0, i], vs[:n_vis].mean(0), what="blockdiag causal mean")
+                _close(lsec[0, :, i], np.full(H, math.log(n_vis)), what="bd causal ln")
+
+
+# ---------------------------------------------------------------------------
+# [xf] ALiBi with scale 0: weights proportional to r^(pos_i - pos_j) with
+# r = exp(-slope_h) over the visible keys -- a geometric series.
+# ---------------------------------------------------------------------------
+def pin_alibi_geometric(orc):
+    r = _rng(4)
+    M, N, H, D = 6, 6, 4, 3
+    q = r.standard_normal((1, M, H, D))
+    k, v = r.standard_normal((1, N, H, D)), r.standard_normal((1, N, H, D))
+    slopes = np.array([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)])
+    out, lse = orc.attention(q, k, v, bias=BIAS_CAUSAL, scale=0.0, alibi=True)
+    for h in range(H):
+        ratio = math.exp(-slopes[h])
+        for i in range(M):
+            w = np.array([ratio ** (i - j) for j in range(i + 1)])
+            z = (1.0 - ratio ** (i + 1)) / (1.0 - ratio)
+            _close(out[0, i, h], (w[:, None] * v[0, :i + 1, h]).sum(0) / z, what="alibi out")
+            _close(lse[0, h, i], math.log(z), what="alibi lse")
+    # non-causal: distance is |pos_i - pos_j| on both sides of the diagonal
+    out, lse = orc.attention(q, k, v, bias=BIAS_NONE, scale=0.0, alibi=True)
+    h, i = 0, 2
+    ratio = math.exp(-slopes[h])
+    w = np.array([ratio ** abs(i - j) for j in range(N)])
+    _close(out[0, i, h], (w[:, None] * v[0, :, h]).sum(0) / w.sum(), what="alibi |i-j|")
+    _close(lse[0, h, i], math.log(w.sum()), what="alibi |i-j| lse")
+
+
+def pin_alibi_slopes(orc):
+    """Slopes 2^(-8(h+1)/Hq): Hq=8 gives 1/2 .. 1/256; Hq=16 interleaves the half steps."""
+    _close(orc.alibi_slopes(8), [2.0 ** -(h + 1) for h in range(8)], what="slopes Hq=8")
+    _close(orc.alibi_slopes(16), [2.0 ** (-(h + 1) / 2.0) for h in range(16)], what="Hq=16")
+    _close(orc.alibi_slopes(1), [2.0 ** -8], what="Hq=1")
+
+
+def pin_alibi_zero_slopes_is_no_bias(orc):
+    r = _rng(5)
+    q, k, v = (r.standard_normal((2, 5, 4, 8)) for _ in range(3))
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        a = orc.attention(q, k, v, bias=bias, alibi=np.zeros(4))
+        b = orc.attention(q, k, v, bias=bias)
+        _close(a[0], b[0], what="alibi 0 out")
+        _close(a[1], b[1], what="alibi 0 lse")
+
+
+# ---------------------------------------------------------------------------
+# Hand-worked cases.
+# ---------------------------------------------------------------------------
+def pin_two_key_hand_case(orc):
+    """q = e0, k0 = 0, k1 = ln(3) e0, scale 1: scores (0, ln 3) -> weights (1/4, 3/4)."""
+    q = np.zeros((1, 1, 1, 2))
+    q[0, 0, 0, 0] = 1.0
+    k = np.zeros((1, 2, 1, 2))
+    k[0, 1, 0, 0] = math.log(3.0)
+    v = np.array([[1.0, 2.0], [5.0, -2.0]]).reshape(1, 2, 1, 2)
+    out, lse = orc.attention(q, k, v, bias=BIAS_NONE, scale=1.0)
+    _close(out[0, 0, 0], [4.0, -1.0], what="hand out")
+    _close(lse[0, 0, 0], math.log(4.0), what="hand lse")
+    # causal with M=1, N=2: the single query sits at position 1 and sees both keys
+    out, _ = orc.attention(q, k, v, bias=BIAS_CAUSAL, scale=1.0)
+    _close(out[0, 0, 0], [4.0, -1.0], what="hand causal bottom-right")
+
+
+def pin_alibi_hand_case(orc):
+    """Hq=2 causal, q.k = 0, row 1: scores (-slope_h, 0); slope_0 = 2^-4, slope_1 = 2^-8."""
+    q = np.zeros((1, 2, 2, 2))
+    k = np.zeros((1, 2, 2, 2))
+    v = np.array([[3.0, 1.0], [-1.0, 2.0]])
+    vv = np.stack([v, v], axis=1).reshape(1, 2, 2, 2)
+    out, lse = orc.attention(q, k, vv, bias=BIAS_CAUSAL, scale=1.0, alibi=True)
+    for h, slope in ((0, 2.0 ** -4), (1, 2.0 ** -8)):
+        e = math.exp(-slope)
+        _close(out[0, 1, h], (e * v[0] + v[1]) / (1.0 + e), what="alibi hand out")
+        _close(lse[0, h, 1], math.log(1.0 + e), what="alibi hand lse")
+
+
+# ---------------------------------------------------------------------------
+# Structural invariants.
+# ---------------------------------------------------------------------------
+def pin_blockdiag_is_independent_runs(orc):
+    """[xf] a packed batch with a block-diagonal mask equals one run per sequence."""
+    r = _rng(6)
+    Hq, Hkv, D = 4, 2, 8
+    lens_q, lens_k = [5, 1, 7, 3], [5, 4, 9, 2]
+    sq, sk = _offsets(lens_q), _offsets(lens_k)
+    q = r.standard_normal((1, sum(lens_q), Hq, D))
+    k, v = r.standard_normal((1, sum(lens_k), Hkv, D)), r.standard_normal((1, sum(lens_k), Hkv, D))
+    for packed_bias, single_bias in ((BIAS_BLOCKDIAG, BIAS_NONE),
+                                     (BIAS_BLOCKDIAG_CAUSAL, BIAS_CAUSAL)):
+        for alibi in (False, True):
+            out, lse = orc.attention(q, k, v, bias=packed_bias, seqstart_q=sq, seqstart_k=sk,
+                                     alibi=alibi)
+            for s in range(len(lens_q)):
+                qs = q[:, sq[s]:sq[s + 1]]
+                ks, vs = k[:, sk[s]:sk[s + 1]], v[:, sk[s]:sk[s + 1]]
+                o1, l1 = orc.attention(qs, ks, vs, bias=single_bias, alibi=alibi)
+                _close(out[:, sq[s]:sq[s + 1]], o1, what=f"blockdiag seq {s}")
+                _close(lse[:, :, sq[s]:sq[s + 1]], l1, what=f"blockdiag lse seq {s}")
+
+
+def pin_gqa_is_repeated_kv(orc):
+    """[xf] query head h reads kv head h // (Hq/Hkv): same as repeating each kv head."""
+    r = _rng(7)
+    B, M, N, Hq, Hkv, D = 2, 5, 6, 8, 2, 4
+    q = r.standard_normal((B, M, Hq, D))
+    k, v = r.standard_normal((B, N, Hkv, D)), r.standard_normal((B, N, Hkv, D))
+    G = Hq // Hkv
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        a = orc.attention(q, k, v, bias=bias, alibi=True)
+        b = orc.attention(q, kr, vr, bias=bias, alibi=True)
+        _close(a[0], b[0], what="gqa out")
+        _close(a[1], b[1], what="gqa lse")
+
+
+def pin_decode_is_last_row(orc):
+    """[decode] one decode step equals the last row of a causal prefill over the
+    same keys, whose last query is the decode query."""
+    r = _rng(8)
+    Hq, Hkv, D = 4, 2, 8
+    lens = [1, 5, 3, 8]
+    st = _offsets(lens)
+    T = int(st[-1])
+    qd = r.standard_normal((len(lens), Hq, D))
+    kc, vc = r.standard_normal((T, Hkv, D)), r.standard_normal((T, Hkv, D))
+    for alibi in (False, True):
+        out, lse = orc.decode(qd, kc, vc, st, scale=0.3, alibi=alibi)
+        for b, n in enumerate(lens):
+            qp = r.standard_normal((1, n, Hq, D))
+            qp[0, n - 1] = qd[b]
+            ks, vs = kc[None, st[b]:st[b + 1]], vc[None, st[b]:st[b + 1]]
+            o, l = orc.attention(qp, ks, vs, bias=BIAS_CAUSAL, scale=0.3, alibi=alibi)
+            _close(out[b], o[0, n - 1], what=f"decode out b={b}")
+            _close(lse[b], l[0, :, n - 1], what=f"decode lse b={b}")
+    # an empty cache sees no key
+    out, lse = orc.decode(qd[:1], kc[:0], vc[:0], np.array([0, 0], dtype=np.int32))
+    _close(out, np.zeros_like(out))
+    assert np.isneginf(lse).all()
+
+
+def pin_key_shift_invariance(orc):
+    """Adding one vector u to every key shifts each score of row i by
+    scale <q_i, u>: out is unchanged and lse moves by that amount."""
+    r = _rng(9)
+    q, k, v = (r.standard_normal((1, 5, 2, 4)) for _ in range(3))
+    u = r.standard_normal(4)
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        a = orc.attention(q, k, v, bias=bias, scale=0.5)
+        b = orc.attention(q, k + u, v, bias=bias, scale=0.5)
+        _close(a[0], b[0], tol=1e-10, what="shift out")
+        _close(b[1] - a[1], 0.5 * np.einsum("bmhd,d->bhm", q, u), tol=1e-10, what="shift lse")
+
+
+def pin_rows_match_full(orc):
+    """The sampled-row entry point returns the same rows as the full one."""
+    r = _rng(10)
+    q = r.standard_normal((2, 6, 4, 8))
+    k, v = r.standard_normal((2, 7, 2, 8)), r.standard_normal((2, 7, 2, 8))
+    rows = np.array([[0, 0, 0], [1, 5, 3], [0, 3, 2], [1, 1, 1]])
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        out, lse = orc.attention(q, k, v, bias=bias, alibi=True)
+        o, l = orc.attention_rows(q, k, v, rows, bias=bias, alibi=True)
+        _close(o, out[rows[:, 0], rows[:, 1], rows[:, 2]], what="rows out")
+        _close(l, lse[rows[:, 0], rows[:, 2], rows[:, 1]], what="rows lse")
+
+
+# ---------------------------------------------------------------------------
+# Brute force: an independent full-matrix formulation with an explicit boolean
+# mask (the form of the "Un cache KV simple" listing), on tiny sizes.
+# ---------------------------------------------------------------------------
+def brute_force(q, k, v, causal, seq_q=None, seq_k=None, slopes=None, scale=None):
+    B, M, Hq, D = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    G = Hq // Hkv
+    if seq_q is None:
+        seq_q, seq_k = [M], [N]
+    qid = np.repeat(np.arange(len(seq_q)), seq_q)
+    kid = np.repeat(np.arange(len(seq_k)), seq_k)
+    qpos = np.concatenate([np.arange(m) + (n - m) for m, n in zip(seq_q, seq_k)])
+    kpos = np.concatenate([np.arange(n) for n in seq_k])
+    allowed = qid[:, None] == kid[None, :]
+    if causal:
+        allowed &= kpos[None, :] <= qpos[:, None]
+    out = np.zeros((B, M, Hq, D))
+    lse = np.full((B, Hq, M), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            S = scale * (q[b, :, h] @ k[b, :, h // G].T)
+            if slopes is not None:
+                S = S - slopes[h] * np.abs(qpos[:, None] - kpos[None, :])
+            S = np.where(allowed, S, -np.inf)
+            for i in range(M):
+                if not allowed[i].any():
+                    continue
+                m = S[i].max()
+                e = np.exp(S[i] - m)
+                out[b, i, h] = (e / e.sum()) @ v[b, :, h // G]
+                lse[b, h, i] = m + math.log(e.sum())
+    return out, lse
+
+
+def pin_brute_force(orc):
+    r = _rng(11)
+    for (B, M, N, Hq, Hkv, D) in ((2, 5, 5, 4, 2, 8), (1, 3, 8, 2, 1, 4), (2, 8, 3, 3, 3, 5)):
+        q = r.standard_normal((B, M, Hq, D))
+        k, v = r.standard_normal((B, N, Hkv, D)), r.standard_normal((B, N, Hkv, D))
+        slopes = orc.alibi_slopes(Hq)
+        for causal in (False, True):
+            for sl in (None, slopes):
+                o, l = orc.attention(q, k, v, bias=BIAS_CAUSAL if causal else BIAS_NONE,
+                                     alibi=sl if sl is not None else None)
+                ob, lb = brute_force(q, k, v, causal, slopes=sl)
+                _close(o, ob, tol=1e-10, what="brute out")
+                _close(l, lb, tol=1e-10, what="brute lse")
+    lens_q, lens_k = [3, 2, 6], [4, 2, 5]
+    q = r.standard_normal((1, 11, 4, 8))
+    k, v = r.standard_normal((1, 11, 2, 8)), r.standard_normal((1, 11, 2, 8))
+    for causal in (False, True):
+        o, l = orc.attention(q, k, v, bias=BIAS_BLOCKDIAG_CAUSAL if causal else BIAS_BLOCKDIAG,
+                             seqstart_q=_offsets(lens_q), seqstart_k=_offsets(lens_k), alibi=True)
+        ob, lb = brute_force(q, k, v, causal, lens_q, lens_k, slopes=orc.alibi_slopes(4))
+        _close(o, ob, tol=1e-10, what="brute varlen out")
+        _close(l, lb, tol=1e-10, what="brute varlen lse")
+
+
+PINS = [
+    pin_weights_sum_to_one,
+    pin_causal_row0_is_v0,
+    pin_scale_zero_means,
+    pin_alibi_geometric,
+    pin_alibi_slopes,
+    pin_alibi_zero_slopes_is_no_bias,
+    pin_two_key_hand_case,
+    pin_alibi_hand_case,
+    pin_blockdiag_is_independent_runs,
+    pin_gqa_is_repeated_kv,
+    pin_decode_is_last_row,
+    pin_key_shift_invariance,
+    pin_rows_match_full,
+    pin_brute_force,
+]
