@@ -1,0 +1,506 @@
+#!/usr/bin/env python
+"""Benchmark: memory-efficient exact attention on B200 through libmea's C ABI.
+
+Headline (one JSON line on rank 0): prefill TFLOP/s on the non-causal sequence
+sweep B=8, H=16, K=64, fp16, M=N in {512, 1024, 2048, 4096} -- one step is one
+mea_fwd call per sequence length.  The same line carries the roofline of the
+prefill kernel, the KV-cache GB/s of a decode step (B=64, cached lengths
+U[512, 8192], Hq=32, Hkv=8, K=128, bf16) with its own roofline, the other
+prefill workloads (packed variable-length causal; GQA + ALiBi causal; the small
+causal example), peak memory against a materialised-score baseline, clocks
+sampled during the timed region, an end-to-end number with host buffers, and
+the fp64 oracle timed on the host cores as a CPU baseline.
+
+FLOPs count only visible (unmasked) query/key pairs: 4 * K * Hq * pairs.
+Decode bytes are the cache rows read once (K and V) plus q and out.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launched by torchrun, each rank runs the same workload on its own
+GPU (independent batches, weak scaling, no data-path collective); time is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "attention TFLOP/s (prefill) and KV-cache GB/s (decode) on 1 B200, % of roofline"
+WORKLOAD = "noncausal_fwd_sweep B=8 H=16 K=64 fp16 M=N in {512,1024,2048,4096}"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "memory_efficient_exact_mea_b200", "csrc")
+
+
+# ---------------------------------------------------------------------------
+# Work accounting
+# ---------------------------------------------------------------------------
+def visible_pairs(M: int, N: int, causal: bool) -> int:
+    if not causal:
+        return M * N
+    off = N - M
+    return sum(max(0, min(N, i + off + 1)) for i in range(M))
+
+
+def prefill_flops(p: synth.Prefill) -> float:
+    causal = p.bias in ("causal", "blockdiag_causal")
+    if p.seq_lens_q is not None:
+        lk = p.seq_lens_k if p.seq_lens_k is not None else p.seq_lens_q
+        pairs = sum(visible_pairs(m, n, causal) for m, n in zip(p.seq_lens_q, lk))
+    else:
+        pairs = p.B * visible_pairs(p.M, p.N, causal)
+    return 4.0 * p.K * p.Hq * pairs
+
+
+def decode_bytes(d: synth.Decode) -> float:
+    el = 2
+    cache = 2.0 * sum(d.kv_lens) * d.Hkv * d.K * el
+    return cache + 2.0 * d.B * d.Hq * d.K * el
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, scale_units: float | None = None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    e = t.get("kernels", {}).get(kernel)
+    return None if e is None else e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], float(parts[3])))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[3] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU; timing reduction only)
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# The measured path
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local):
+    import memory_efficient_exact_mea_b200 as mea
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peaks_kind = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])  # fp16 and bf16 share the nominal dense rate
+
+    # ---- headline workload: the sweep --------------------------------------
+    sweep = [synth.noncausal_sweep(M) for M in synth.SWEEP_M]
+    dev_in = [(p.q.to(dev), p.k.to(dev), p.v.to(dev)) for p in sweep]
+    outs = [torch.empty_like(q) for (q, _, _) in dev_in]
+    lses = [torch.empty((p.B, p.Hq, p.M), dtype=torch.float32, device=dev) for p in sweep]
+    flops = [prefill_flops(p) for p in sweep]
+
+    def step(events=None):
+        for i, (p, (q, k, v)) in enumerate(zip(sweep, dev_in)):
+            if events is not None:
+                events[i][0].record(stream)
+            mea.mea_fwd(q, k, v, bias="none", scale=p.scale, out=outs[i], lse=lses[i])
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert mea.read_device_status() == 0
+
+    per_launch = [[] for _ in sweep]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in sweep]
+               for _ in range(args.steps)]
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    for s in range(args.steps):
+        for i in range(len(sweep)):
+            per_launch[i].append(evs[s][i][0].elapsed_time(evs[s][i][1]))
+    clocks = clk.summary()
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    ms_per_step = elapsed_ms / args.steps
+    total_flops = sum(flops) * args.steps * world
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+
+    kernel_ms = [statistics.mean(x) for x in per_launch]
+    achieved = sum(flops) / (sum(kernel_ms) * 1e-3) / 1e12
+    sweep_detail = []
+    for p, f, ms in zip(sweep, flops, kernel_ms):
+        sweep_detail.append({"M": p.M, "ms": round(ms, 4), "tflops": round(f / ms / 1e9, 1)})
+
+    # ---- peak memory vs a materialised-score baseline (context) ------------
+    if rank == 0 and not args.no_memory:
+        for d, p, (q, k, v) in zip(sweep_detail, sweep, dev_in):
+            d.update(memory_report(mea, p, q, k, v, dev))
+
+    # ---- end to end: host buffers through the public call ------------------
+    e2e = measure_e2e(mea, sweep, dev, stream, args, world)
+
+    # ---- the other workloads (secondary measurements) -----------------------
+    also = {}
+    if not args.quick:
+        also["varlen_causal"] = measure_prefill(mea, synth.varlen_causal(), dev, stream, tc_peak)
+        also["gqa_alibi_causal"] = measure_prefill(mea, synth.gqa_alibi_causal(), dev, stream,
+                                                   tc_peak)
+        also["causal_small"] = measure_prefill(mea, synth.causal_small(), dev, stream, tc_peak,
+                                               iters=50)
+        also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
+    assert mea.read_device_status() == 0
+
+    traffic = traffic_for("fwd_kernel<64,f16,none>")
+    roofline = {
+        "kernel": "fwd_kernel<K=64,f16,no mask> (sweep launches)",
+        "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
+        "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+        "peak_kind": f"{peaks_kind} bf16 burst (fp16 nominal rate = bf16)",
+        "traffic": traffic,
+        "algorithmic": "4*K*H*B*M*N FLOP per launch",
+    }
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": 8, "H": 16, "K": 64, "seq_lens": list(synth.SWEEP_M),
+                   "bias": "none", "global_batch": 8 * world,
+                   "l2": "inputs exceed L2: 502 MB read per step in a fixed order",
+                   "parallelism": f"replica x{world}"},
+        "roofline": roofline, "sweep": sweep_detail, "also": also, "e2e": e2e,
+        "gpu_launches": len(sweep) * args.steps, "clocks": clocks,
+        "impl": "ours",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(sweep[-1], args.cpu_seconds)
+    return line
+
+
+def memory_report(mea, p, q, k, v, dev):
+    """Peak device MB of one call: ours vs the plain materialised-score attention."""
+    torch.cuda.synchronize(dev)
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    out, lse = mea.mea_fwd(q, k, v, scale=p.scale)
+    torch.cuda.synchronize(dev)
+    ours = (torch.cuda.max_memory_allocated(dev) - base) / 1e6
+    del out, lse
+    torch.cuda.synchronize(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    # Materialised scores (the pages' naive attention), [B, H, M, N] in fp16.
+    qt, kt, vt = (x.permute(0, 2, 1, 3) for x in (q, k, v))
+
+    def naive():
+        s = torch.matmul(qt, kt.transpose(-1, -2)) * p.scale
+        return torch.matmul(torch.softmax(s, dim=-1), vt)
+
+    naive()
+    torch.cuda.synchronize(dev)
+    naive_mb = (torch.cuda.max_memory_allocated(dev) - base) / 1e6
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        naive()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    return {"peak_mb_ours": round(ours, 1), "peak_mb_materialised": round(naive_mb, 1),
+            "scores_mb_analytic": round(p.B * p.Hq * p.M * p.N * 2 / 1e6, 1),
+            "materialised_ms": round(e0.elapsed_time(e1) / 3, 3)}
+
+
+def measure_e2e(mea, sweep, dev, stream, args, world):
+    """Same metric through the public call with host buffers: pinned H2D of q,k,v,
+    the kernel, D2H of out and lse, every step, inside the timed region."""
+    host = [(p.q.pin_memory(), p.k.pin_memory(), p.v.pin_memory()) for p in sweep]
+    dbuf = [(torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev),
+             torch.empty_like(hv, device=dev)) for (hq, hk, hv) in host]
+    houts = [torch.empty_like(p.q).pin_memory() for p in sweep]
+    hlses = [torch.empty((p.B, p.Hq, p.M), dtype=torch.float32).pin_memory() for p in sweep]
+    dout = [torch.empty_like(d[0]) for d in dbuf]
+    dlse = [torch.empty((p.B, p.Hq, p.M), dtype=torch.float32, device=dev) for p in sweep]
+    h2d = sum(x.numel() * x.element_size() for t in host for x in t)
+    d2h = sum(x.numel() * x.element_size() for x in houts) + sum(
+        x.numel() * x.element_size() for x in hlses)
+
+    def step():
+        for i, p in enumerate(sweep):
+            for dst, src in zip(dbuf[i], host[i]):
+                dst.copy_(src, non_blocking=True)
+            mea.mea_fwd(*dbuf[i], scale=p.scale, out=dout[i], lse=dlse[i])
+            houts[i].copy_(dout[i], non_blocking=True)
+            hlses[i].copy_(dlse[i], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    n = max(1, min(args.steps, 5))
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    flops = sum(prefill_flops(p) for p in sweep) * n * world
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "ms_per_step": round(ms / n, 3)}
+
+
+def _time(fn, stream, iters, warmup=3):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def measure_prefill(mea, p, dev, stream, tc_peak, iters=10):
+    q, k, v = p.q.to(dev), p.k.to(dev), p.v.to(dev)
+    kw = {}
+    if p.seq_lens_q is not None:
+        kw = dict(seqstart_q=p.seqstart_q.to(dev), seqstart_k=p.seqstart_k.to(dev),
+                  max_seqlen_q=max(p.seq_lens_q),
+                  max_seqlen_k=max(p.seq_lens_k or p.seq_lens_q))
+    out = torch.empty_like(q)
+    lse = torch.empty((p.B, p.Hq, p.M), dtype=torch.float32, device=dev)
+    ms = _time(lambda: mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, out=out,
+                                   lse=lse, **kw), stream, iters)
+    f = prefill_flops(p)
+    tf = f / (ms * 1e-3) / 1e12
+    return {"workload": p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
+            "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor"}
+
+
+def measure_decode(mea, d, dev, stream, hbm_peak, iters=20):
+    q, kc, vc = d.q.to(dev), d.k_cache.to(dev), d.v_cache.to(dev)
+    st = d.kv_seqstart.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((d.B, d.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(mea.mea_decode_workspace_size(d.B, d.Hq, d.Hkv, d.K, d.max_kv_len),
+                     dtype=torch.uint8, device=dev)
+    ms = _time(lambda: mea.mea_decode(q, kc, vc, st, d.max_kv_len, scale=d.scale, out=out, lse=lse,
+                                      workspace=ws), stream, iters)
+    nbytes = decode_bytes(d)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": d.name, "ms": round(ms, 4), "gbs": round(gbs, 1),
+            "frac": round(gbs / hbm_peak, 4), "bytes": nbytes, "bound": "hbm",
+            "peak": hbm_peak, "note": "cache larger than L2 (1.1 GB)"}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on the host cores, bounded sample
+# ---------------------------------------------------------------------------
+def cpu_baseline(p: synth.Prefill, seconds: float):
+    import oracle
+
+    orc = oracle.get()
+    qf = p.q.to(torch.float64).numpy()
+    kf = p.k.to(torch.float64).numpy()
+    vf = p.v.to(torch.float64).numpy()
+    rng = np.random.default_rng(0)
+    rows_done, t_used, batch = 0, 0.0, 64
+    while t_used < seconds:
+        rows = np.stack([rng.integers(p.B, size=batch), rng.integers(p.M, size=batch),
+                         rng.integers(p.Hq, size=batch)], axis=1)
+        t = time.perf_counter()
+        orc.attention_rows(qf, kf, vf, rows, bias=0, scale=p.scale)
+        t_used += time.perf_counter() - t
+        rows_done += batch
+        batch = min(batch * 2, 4096)
+    flops = rows_done * 4.0 * p.K * p.N
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(flops / t_used / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{rows_done} random query rows of M=N={p.M} (B=8,H=16,K=64) in "
+                      f"{t_used:.1f} s, fp64 C oracle, OpenMP over rows"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm for this build is the fp64 oracle on the host cores."""
+    if rank != 0:
+        return None
+    p = synth.noncausal_sweep(4096)
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(p, per_step / 4)
+    vals = [cpu_baseline(p, per_step) for _ in range(args.steps)]
+    v = statistics.mean(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = round(v, 6)
+    return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": 8, "H": 16, "K": 64,
+                       "seq_lens": list(synth.SWEEP_M), "bias": "none"},
+            "impl": "reference", "cpu_baseline": cb,
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline only, skip other workloads")
+    ap.add_argument("--no-memory", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

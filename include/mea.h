@@ -1,0 +1,166 @@
+/*
+ * mea.h -- C ABI of libmea: memory-efficient exact attention on B200 (sm_100a).
+ *
+ * The operation (FlashAttention (2022), sections "L'idea: non scrivere mai la
+ * matrice intera" and "Il trucco della softmax che non ha bisogno di vedere
+ * tutto"; xFormers tutorial "Come costruire Transformer efficienti in memoria
+ * con xFormers ...", section "Impostare xFormers e Validare l'Attenzione
+ * Memory-Efficient"):
+ *
+ *     out = softmax(Q K^T * scale + bias) V,   lse = ln sum_j exp(scale q.k_j + b_j)
+ *
+ * computed tile by tile with a running max / running sum, so the M x N score
+ * matrix never reaches device memory.  The result is exact up to the rounding of
+ * fp32 accumulation and of the fp16/bf16 output.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates nothing, keeps no pointer after the call returns and is safe to
+ *    call from several host threads.
+ *  - Calls are asynchronous on `stream` and never synchronise (except
+ *    mea_read_device_status).  Argument errors are detected on the host and
+ *    returned before anything is launched; nothing is thrown across the ABI.
+ *  - Element types: MEA_F16 or MEA_BF16 for q/k/v/out; lse is fp32.
+ *    Accumulation is fp32 throughout.
+ *  - Head dimension K must be 64 or 128.  Base pointers must be 16-byte aligned
+ *    and every stride a multiple of 8 elements (tensor-memory-accelerator
+ *    copies require 16-byte aligned rows); otherwise MEA_ERR_UNSUPPORTED.
+ *  - Contents of device-side index arrays (seqstart offsets) are trusted; a
+ *    kernel that finds them inconsistent with the host-side sizes records
+ *    MEA_ERR_INVALID_ARG in the device status word (see
+ *    mea_read_device_status) instead of faulting.
+ *  - Every device wait is bounded: a wait that exceeds about two seconds makes
+ *    the kernel record MEA_ERR_DEVICE_TIMEOUT and return, never hang.
+ */
+#ifndef MEA_H_
+#define MEA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MEA_F16 = 0, MEA_BF16 = 1 } mea_dtype_t;
+
+/* The bias objects of the xFormers tutorial, as an enum: the masks are
+ * generated inside the kernel, never stored ("Applicare Attenzione Causale con
+ * Maschere Inferiori"; "Utilizzare Sequenze di Lunghezza Variabile"). */
+typedef enum {
+  MEA_BIAS_NONE = 0,             /* no mask                                  */
+  MEA_BIAS_CAUSAL = 1,           /* LowerTriangularMask, bottom-right aligned */
+  MEA_BIAS_BLOCKDIAG = 2,        /* BlockDiagonalMask over packed sequences   */
+  MEA_BIAS_BLOCKDIAG_CAUSAL = 3  /* BlockDiagonalCausalMask                   */
+} mea_bias_t;
+
+typedef enum {
+  MEA_OK = 0,
+  MEA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, inconsistent shapes     */
+  MEA_ERR_UNSUPPORTED = -2,   /* valid but not implemented (K, alignment, dtype) */
+  MEA_ERR_WORKSPACE = -3,     /* workspace missing or too small                  */
+  MEA_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed               */
+  MEA_ERR_DEVICE_TIMEOUT = -5 /* a bounded device wait ran out (device status)   */
+} mea_status_t;
+
+/*
+ * mea_fwd -- prefill / training-forward attention.
+ *
+ * Layouts (element strides; the last dimension K is contiguous):
+ *   q   [B, M, Hq,  K]  q_strides = {stride_b, stride_m, stride_h}
+ *   k   [B, N, Hkv, K]  k_strides
+ *   v   [B, N, Hkv, K]  v_strides
+ *   out [B, M, Hq,  K]  o_strides  (written; same dtype as q)
+ *   lse [B, Hq, M] fp32, contiguous, natural log; may be NULL.
+ *
+ * Heads: Hq % Hkv == 0; query head h reads key/value head h / (Hq / Hkv)
+ * (grouped-query attention, tutorial section "Dimotrazione di Gruppo Query
+ * Attention (GQA)"), without copying K/V.
+ *
+ * bias:
+ *   NONE    every query sees every key.
+ *   CAUSAL  query i sees key j iff j <= i + (N - M) (bottom-right alignment, the
+ *           tril(diagonal=past_len) mask of "Transformer : comprendre
+ *           l'entrainement et l'inference", section "Un cache KV simple").
+ *   BLOCKDIAG / BLOCKDIAG_CAUSAL  packed variable-length batch: B must be 1 and
+ *           seqstart_q / seqstart_k (DEVICE int32 arrays of num_seqs + 1
+ *           non-decreasing offsets, first 0, last M resp. N) split the rows into
+ *           sequences; a query sees only keys of its own sequence, and with
+ *           _CAUSAL the bottom-right rule applies inside the sequence.
+ *           seqstart_k may be NULL (then equal to seqstart_q, requires M == N).
+ *           max_seqlen_q / max_seqlen_k are host-known upper bounds on the
+ *           per-sequence lengths (they size the grid; no device sync is made).
+ *           For NONE / CAUSAL pass NULL, NULL, 0, 0, 0.
+ * alibi:  nonzero adds -slope_h * |pos_i - pos_j| after scaling, positions local
+ *         to the sequence with pos_i = i + (N - M), slope_h = 2^(-8 (h+1) / Hq)
+ *         computed in registers (tutorial section "Utilizzare SwiGLU e ALiBi").
+ * scale:  multiplies q.k (pass 1/sqrt(K) for the usual attention).
+ *
+ * A query row that sees no key gets out = 0 and lse = -inf.
+ * Returns MEA_OK or an error status; never synchronises.
+ */
+int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+            int B, int M, int N, int Hq, int Hkv, int K,
+            const int64_t q_strides[3], const int64_t k_strides[3],
+            const int64_t v_strides[3], const int64_t o_strides[3],
+            mea_dtype_t dtype, mea_bias_t bias,
+            const int32_t* seqstart_q, const int32_t* seqstart_k,
+            int num_seqs, int max_seqlen_q, int max_seqlen_k,
+            int alibi, float scale, cudaStream_t stream);
+
+/*
+ * mea_decode -- one decode step: a single new query per sequence against a
+ * packed, ragged KV cache ("Transformer : comprendre l'entrainement et
+ * l'inference", section "Pre-remplissage et decodage"; "Transformerを実装して
+ * 少し理解した気になる会(その4)", section "KV Cache": only the last query row is
+ * needed, against every cached key).
+ *
+ *   q        [B, Hq, K]       contiguous (a [B, 1, Hq, K] tensor)
+ *   k_cache  [cache_rows, Hkv, K] contiguous; v_cache the same
+ *   kv_seqstart  DEVICE int32 [B + 1]: sequence b owns cache rows
+ *            kv_seqstart[b] .. kv_seqstart[b+1]-1 (its keys, oldest first,
+ *            the new token's key/value already appended); kv_seqstart[B] <= cache_rows.
+ *   out      [B, Hq, K]       written, same dtype as q
+ *   lse      [B, Hq] fp32 natural log, may be NULL
+ *   max_kv_len  host-known upper bound on every n_b (sizes the split grid).
+ *
+ * The query of sequence b sits at position n_b - 1 and sees all n_b keys
+ * (with ALiBi: bias -slope_h * (n_b - 1 - j)).  An empty sequence gives out = 0,
+ * lse = -inf.  The cache is split into fixed chunks processed in parallel; the
+ * partial (max, sum, output) states are merged exactly by their log-sum-exp.
+ *
+ * workspace: DEVICE scratch of at least mea_decode_workspace_size(...) bytes,
+ * 256-byte aligned, owned by the caller; its contents need no initialisation
+ * and are garbage afterwards.  Calls that share a workspace must not overlap.
+ */
+size_t mea_decode_workspace_size(int B, int Hq, int Hkv, int K, int max_kv_len);
+
+int mea_decode(const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* kv_seqstart, void* out, float* lse,
+               int B, int Hq, int Hkv, int K, int cache_rows, int max_kv_len,
+               mea_dtype_t dtype, int alibi, float scale,
+               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of key/value rows one decode split covers (the unit of parallelism). */
+int mea_decode_chunk(void);
+
+/* Text for a status code (static storage; never NULL). */
+const char* mea_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns the first error a kernel recorded in the
+ * current device's status word (MEA_OK if none) and, if `clear` is nonzero,
+ * resets it to MEA_OK.  Returns MEA_ERR_CUDA if the synchronisation fails.
+ */
+int mea_read_device_status(cudaStream_t stream, int clear);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mea_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEA_H_ */

@@ -1,0 +1,186 @@
+"""memory_efficient_exact_mea_b200 -- memory-efficient exact attention on B200.
+
+A thin ctypes binding of ``libmea.so`` (C ABI in ``include/mea.h``).  This module
+only marshals arguments: every step of the computation runs in the library's
+sm_100a kernels.  PyTorch supplies device memory and the current stream.  There
+is no fallback: importing this package fails loudly if ``libmea.so`` is missing.
+
+Operations (sources cited in ``include/mea.h``):
+  mea_fwd     softmax(Q K^T * scale + bias) V and the per-row log-sum-exp, with
+              no / causal / block-diagonal (causal) masks, GQA and ALiBi.
+  mea_decode  one query per sequence against a packed, ragged KV cache.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["mea_fwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
+           "read_device_status", "status_string", "MeaError", "BIAS", "LIB_PATH", "lib"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
+
+BIAS = {"none": 0, "causal": 1, "blockdiag": 2, "blockdiag_causal": 3}
+_DTYPE = {torch.float16: 0, torch.bfloat16: 1}
+_i64x3 = ctypes.c_int64 * 3
+
+
+class MeaError(RuntimeError):
+    """A libmea entry point returned an error status."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m memory_efficient_exact_mea_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.mea_fwd.restype = i
+    L.mea_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, i, i, vp, vp,
+                          i, i, i, i, f, vp]
+    L.mea_decode_workspace_size.restype = sz
+    L.mea_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.mea_decode.restype = i
+    L.mea_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.mea_decode_chunk.restype = i
+    L.mea_decode_chunk.argtypes = []
+    L.mea_status_string.restype = ctypes.c_char_p
+    L.mea_status_string.argtypes = [i]
+    L.mea_read_device_status.restype = i
+    L.mea_read_device_status.argtypes = [vp, i]
+    L.mea_version.restype = i
+    L.mea_version.argtypes = []
+    return L
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.mea_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MeaError(fn, rc)
+
+
+def _bmhk_strides(t: torch.Tensor, name: str):
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, rows, heads, K]")
+    if t.stride(3) != 1:
+        raise ValueError(f"{name}: the last dimension must be contiguous")
+    return _i64x3(t.stride(0), t.stride(1), t.stride(2))
+
+
+def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool = False,
+            seqstart_q=None, seqstart_k=None, max_seqlen_q: int | None = None,
+            max_seqlen_k: int | None = None, out=None, lse=None, return_lse: bool = True,
+            stream=None):
+    """Attention forward.  q [B,M,Hq,K], k/v [B,N,Hkv,K] (fp16/bf16, CUDA) ->
+    (out [B,M,Hq,K], lse [B,Hq,M] fp32 or None).
+
+    bias: "none" | "causal" | "blockdiag" | "blockdiag_causal".  The block-diagonal
+    kinds take B == 1 and int32 CUDA offsets ``seqstart_q`` (and ``seqstart_k``);
+    ``max_seqlen_q`` is the longest query sequence (read from the offsets, with a
+    device-to-host copy, when not given).
+    """
+    B, M, Hq, K = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    if q.dtype not in _DTYPE or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype float16 or bfloat16")
+    if tuple(k.shape) != (B, N, Hkv, K) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, N, Hkv, K]")
+    scale = K ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, M, Hq, K), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, M), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, Hq, M] tensor")
+    kind = BIAS[bias]
+    ns = 0
+    if kind >= 2:
+        if seqstart_q is None:
+            raise ValueError("block-diagonal bias needs seqstart_q")
+        for s in (seqstart_q, seqstart_k):
+            if s is not None and (s.dtype != torch.int32 or not s.is_cuda):
+                raise ValueError("seqstart offsets must be int32 CUDA tensors")
+        ns = seqstart_q.numel() - 1
+        if max_seqlen_q is None:
+            max_seqlen_q = int(torch.diff(seqstart_q).max().item()) if ns > 0 else 0
+        if max_seqlen_k is None:
+            sk = seqstart_q if seqstart_k is None else seqstart_k
+            max_seqlen_k = int(torch.diff(sk).max().item()) if ns > 0 else 0
+    else:
+        seqstart_q = seqstart_k = None
+        max_seqlen_q = max_seqlen_k = 0
+    rc = lib.mea_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, M, N, Hq, Hkv, K,
+                     _bmhk_strides(q, "q"), _bmhk_strides(k, "k"), _bmhk_strides(v, "v"),
+                     _bmhk_strides(out, "out"), _DTYPE[q.dtype], kind, _ptr(seqstart_q),
+                     _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k), int(bool(alibi)),
+                     scale, _stream(stream))
+    _check("mea_fwd", rc)
+    return out, lse
+
+
+def mea_decode_workspace_size(B: int, Hq: int, Hkv: int, K: int, max_kv_len: int) -> int:
+    return int(lib.mea_decode_workspace_size(B, Hq, Hkv, K, max_kv_len))
+
+
+def mea_decode_chunk() -> int:
+    return int(lib.mea_decode_chunk())
+
+
+def mea_decode(q, k_cache, v_cache, kv_seqstart, max_kv_len: int, scale: float | None = None,
+               alibi: bool = False, out=None, lse=None, workspace=None, return_lse: bool = True,
+               stream=None):
+    """One decode step.  q [B,Hq,K] or [B,1,Hq,K]; caches [T,Hkv,K]; kv_seqstart int32
+    CUDA [B+1] -> (out shaped like q, lse [B,Hq] fp32 or None)."""
+    qshape = tuple(q.shape)
+    q3 = q.reshape(q.shape[0], q.shape[-2], q.shape[-1])
+    B, Hq, K = q3.shape
+    T, Hkv = k_cache.shape[0], k_cache.shape[1]
+    for name, t in (("q", q3), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or k_cache.shape[2] != K:
+        raise ValueError("caches must be [T, Hkv, K]")
+    if q.dtype not in _DTYPE or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("q and caches must share dtype float16 or bfloat16")
+    if kv_seqstart.dtype != torch.int32 or not kv_seqstart.is_cuda:
+        raise ValueError("kv_seqstart must be an int32 CUDA tensor")
+    scale = K ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(qshape, dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = mea_decode_workspace_size(B, Hq, Hkv, K, max_kv_len)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.mea_decode(_ptr(q3), _ptr(k_cache), _ptr(v_cache), _ptr(kv_seqstart), _ptr(out),
+                        _ptr(lse), B, Hq, Hkv, K, T, int(max_kv_len), _DTYPE[q.dtype],
+                        int(bool(alibi)), scale, _ptr(workspace), ws_bytes, _stream(stream))
+    _check("mea_decode", rc)
+    return out, lse
+
+
+def read_device_status(clear: bool = True, stream=None) -> int:
+    """Synchronise and return the first error a kernel recorded on this device (0 = none)."""
+    return int(lib.mea_read_device_status(_stream(stream), int(bool(clear))))

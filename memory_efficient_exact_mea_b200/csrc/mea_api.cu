@@ -1,0 +1,253 @@
+// mea_api.cu -- the C ABI declared in include/mea.h: host-side validation,
+// TMA descriptor encoding and kernel dispatch.  No allocation, no global mutable
+// host state (the driver entry point is resolved once, thread-safely).
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "mea.h"
+#include "mea_internal.h"
+
+// First error recorded by a kernel of this library (one word per device).
+__device__ int g_mea_status = 0;
+
+namespace {
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int* status_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_mea_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A [batch, rows, heads, K] tensor with element strides {sb, sm, sh} as a rank-4
+// TMA map (innermost first), 64-element x 1 head x `box_rows` boxes, 128-byte
+// swizzle.  Returns false if the driver rejects it.
+bool encode_bmhk(CUtensorMap* map, const void* base, bool bf16, int batch, int rows, int heads,
+                 int K, const int64_t st[3], int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st[2]) * 2,
+                                 static_cast<cuuint64_t>(st[1]) * 2,
+                                 static_cast<cuuint64_t>(st[0]) * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A packed cache [rows, heads, K] (contiguous) as a rank-3 TMA map.
+bool encode_cache(CUtensorMap* map, const void* base, bool bf16, int rows, int heads, int K,
+                  int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2,
+                                 static_cast<cuuint64_t>(heads) * K * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                  3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool strides_ok(const int64_t s[3]) {
+  for (int i = 0; i < 3; ++i)
+    if (s[i] <= 0 || (s[i] & 7) != 0 || s[i] >= (int64_t(1) << 38)) return false;
+  return true;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int decode_splits(int max_kv_len) {
+  return max_kv_len <= 0 ? 0 : (max_kv_len + mea::kDecodeChunk - 1) / mea::kDecodeChunk;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mea_version(void) { return kVersion; }
+
+const char* mea_status_string(int status) {
+  switch (status) {
+    case MEA_OK: return "ok";
+    case MEA_ERR_INVALID_ARG: return "invalid argument";
+    case MEA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MEA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MEA_ERR_CUDA: return "CUDA error";
+    case MEA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int mea_decode_chunk(void) { return mea::kDecodeChunk; }
+
+int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int M,
+            int N, int Hq, int Hkv, int K, const int64_t q_strides[3], const int64_t k_strides[3],
+            const int64_t v_strides[3], const int64_t o_strides[3], mea_dtype_t dtype,
+            mea_bias_t bias, const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+            int max_seqlen_q, int max_seqlen_k, int alibi, float scale, cudaStream_t stream) {
+  (void)max_seqlen_k;
+  if (B < 0 || M < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return MEA_ERR_INVALID_ARG;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
+  if (bias < MEA_BIAS_NONE || bias > MEA_BIAS_BLOCKDIAG_CAUSAL) return MEA_ERR_INVALID_ARG;
+  if (!q_strides || !k_strides || !v_strides || !o_strides) return MEA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return MEA_ERR_INVALID_ARG;  // NaN
+  if (B == 0 || M == 0) return MEA_OK;
+  if (!q || !out || (N > 0 && (!k || !v))) return MEA_ERR_INVALID_ARG;
+  if (K != 64 && K != 128) return MEA_ERR_UNSUPPORTED;
+  const bool packed = bias == MEA_BIAS_BLOCKDIAG || bias == MEA_BIAS_BLOCKDIAG_CAUSAL;
+  if (packed) {
+    if (B != 1 || !seqstart_q || num_seqs <= 0 || max_seqlen_q < 0) return MEA_ERR_INVALID_ARG;
+    if (!seqstart_k && M != N) return MEA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(out) || (N > 0 && (!aligned16(k) || !aligned16(v))))
+    return MEA_ERR_UNSUPPORTED;
+  if (!strides_ok(q_strides) || !strides_ok(o_strides) ||
+      (N > 0 && (!strides_ok(k_strides) || !strides_ok(v_strides))))
+    return MEA_ERR_UNSUPPORTED;
+
+  int* status = status_word();
+  if (!status) return MEA_ERR_CUDA;
+
+  if (N == 0) {  // no key anywhere: every row is empty
+    return mea::launch_fill_empty(out, lse, B, M, Hq, K, o_strides[0], o_strides[1],
+                                  o_strides[2], stream) == cudaSuccess
+               ? MEA_OK
+               : MEA_ERR_CUDA;
+  }
+
+  mea::FwdLaunch L{};
+  const bool bf16 = dtype == MEA_BF16;
+  if (!encode_bmhk(&L.tmQ, q, bf16, B, M, Hq, K, q_strides, 128) ||
+      !encode_bmhk(&L.tmK, k, bf16, B, N, Hkv, K, k_strides, 128) ||
+      !encode_bmhk(&L.tmV, v, bf16, B, N, Hkv, K, v_strides, 128))
+    return MEA_ERR_CUDA;
+  mea::FwdArgs& a = L.args;
+  a.out = out;
+  a.lse = lse;
+  a.seqstart_q = packed ? seqstart_q : nullptr;
+  a.seqstart_k = packed ? (seqstart_k ? seqstart_k : seqstart_q) : nullptr;
+  a.status = status;
+  a.o_sb = o_strides[0];
+  a.o_sm = o_strides[1];
+  a.o_sh = o_strides[2];
+  a.B = B;
+  a.M = M;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.num_units = packed ? num_seqs : B;
+  const int rows = packed ? max_seqlen_q : M;
+  a.num_mblocks = (rows + mea::kFwdRowsPerCta - 1) / mea::kFwdRowsPerCta;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  L.head_dim = K;
+  L.bf16 = bf16;
+  L.mask = static_cast<int>(bias);
+  L.alibi = alibi != 0;
+  if (a.num_mblocks == 0) return MEA_OK;
+  return mea::launch_fwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+size_t mea_decode_workspace_size(int B, int Hq, int Hkv, int K, int max_kv_len) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || K <= 0 || max_kv_len < 0) return 0;
+  const size_t splits = static_cast<size_t>(decode_splits(max_kv_len));
+  const size_t rows = static_cast<size_t>(B) * Hq * splits;
+  return align256(rows * K * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+int mea_decode(const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* kv_seqstart, void* out, float* lse, int B, int Hq, int Hkv, int K,
+               int cache_rows, int max_kv_len, mea_dtype_t dtype, int alibi, float scale,
+               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || cache_rows < 0 || max_kv_len < 0)
+    return MEA_ERR_INVALID_ARG;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return MEA_ERR_INVALID_ARG;
+  if (B == 0) return MEA_OK;
+  if (!q || !out || !kv_seqstart) return MEA_ERR_INVALID_ARG;
+  if (cache_rows > 0 && (!k_cache || !v_cache)) return MEA_ERR_INVALID_ARG;
+  if (K != 64 && K != 128) return MEA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8) return MEA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(out) ||
+      (cache_rows > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return MEA_ERR_UNSUPPORTED;
+  const size_t need = mea_decode_workspace_size(B, Hq, Hkv, K, max_kv_len);
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return MEA_ERR_WORKSPACE;
+
+  int* status = status_word();
+  if (!status) return MEA_ERR_CUDA;
+
+  mea::DecodeLaunch L{};
+  const bool bf16 = dtype == MEA_BF16;
+  mea::DecodeArgs& a = L.args;
+  a.q = q;
+  a.out = out;
+  a.lse = lse;
+  a.kv_seqstart = kv_seqstart;
+  a.status = status;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.cache_rows = cache_rows;
+  a.max_splits = cache_rows > 0 ? decode_splits(max_kv_len) : 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * decode_splits(max_kv_len);
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                        align256(rows * K * sizeof(float)));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  L.head_dim = K;
+  L.bf16 = bf16;
+  L.alibi = alibi != 0;
+  if (a.max_splits > 0) {
+    if (!encode_cache(&L.tmK, k_cache, bf16, cache_rows, Hkv, K, 64) ||
+        !encode_cache(&L.tmV, v_cache, bf16, cache_rows, Hkv, K, 64))
+      return MEA_ERR_CUDA;
+  }
+  return mea::launch_decode(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+int mea_read_device_status(cudaStream_t stream, int clear) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MEA_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpyFromSymbol(&value, g_mea_status, sizeof(int)) != cudaSuccess)
+    return MEA_ERR_CUDA;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_mea_status, &zero, sizeof(int)) != cudaSuccess) return MEA_ERR_CUDA;
+  }
+  return value;
+}
+
+}  // extern "C"

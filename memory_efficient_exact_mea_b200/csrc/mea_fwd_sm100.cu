@@ -1,0 +1,461 @@
+// mea_fwd_sm100.cu -- prefill attention for B200 (sm_100a): TMA + tcgen05 + TMEM.
+//
+// Computes out = softmax(Q K^T * scale + bias) V and lse per row, tile by tile
+// with a running max and running sum, so the score matrix lives only in tensor
+// memory, one 128x128 tile at a time ("FlashAttention (2022)", sections "L'idea:
+// non scrivere mai la matrice intera" and "Il trucco della softmax che non ha
+// bisogno di vedere tutto").  Masks (causal, block-diagonal) are generated from
+// indices and fully masked key tiles are never loaded ("Come costruire
+// Transformer efficienti in memoria con xFormers ...", "Applicare Attenzione
+// Causale con Maschere Inferiori", "Utilizzare Sequenze di Lunghezza Variabile").
+//
+// CTA organisation (320 threads, one CTA per SM):
+//   warps 0-3  softmax / rescale / epilogue for query tile 0 (TMEM lanes 0-127)
+//   warps 4-7  the same for query tile 1 (rows +128)
+//   warp  8    TMEM allocator and the single MMA-issuing thread
+//   warp  9    the single TMA-issuing thread
+// Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
+// current key tile; P = exp(S - m) in fp16/bf16 is written back over the first
+// 64 columns and fed to the P.V MMA straight from TMEM) | O0 | O1 (K columns
+// each, the fp32 output accumulators).
+// Shared memory: Q0, Q1 (loaded once) and a ring of key/value tiles, all in the
+// 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
+#include <math.h>
+
+#include "mea_internal.h"
+#include "sm100.cuh"
+
+namespace mea {
+namespace {
+
+constexpr int kBM = 128;        // query rows per tile (= TMEM lanes)
+constexpr int kBN = 128;        // keys per tile
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceeds it by < 2^8
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct Smem {
+  static constexpr int kChunks = D / 64;          // 64-element (128-byte) column chunks
+  static constexpr int kChunkBytes = kBM * 128;   // one chunk of a 128-row tile
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kQ = 0;
+  static constexpr int kKV = 2 * kTileBytes;
+  static constexpr int kBar = kKV + kSlots * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
+};
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+template <int D, bool BF16, int MASK, bool ALIBI>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using L = Smem<D>;
+  constexpr bool kCausal = (MASK == 1 || MASK == 3);
+  constexpr bool kPacked = (MASK >= 2);
+  constexpr int S = L::kSlots;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sKV = smem + L::kKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + S;
+  uint64_t* s_full = bars + 1 + 2 * S;
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_done = p_ready + 2;
+  uint64_t* mma_done = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- which (query block, head, batch or sequence) this CTA owns ----------
+  const int per_mb = a.Hq * a.num_units;
+  int mb = blockIdx.x / per_mb;
+  const int rem = blockIdx.x - mb * per_mb;
+  const int h = rem % a.Hq;
+  const int unit = rem / a.Hq;
+  if (kCausal) mb = a.num_mblocks - 1 - mb;  // longest key ranges first
+  const int kvh = h / a.group;
+
+  int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, bidx = unit;
+  if constexpr (kPacked) {
+    q0 = a.seqstart_q[unit];
+    q_len = a.seqstart_q[unit + 1] - q0;
+    k0 = a.seqstart_k[unit];
+    k_len = a.seqstart_k[unit + 1] - k0;
+    bidx = 0;
+    const bool bad = q_len < 0 || k_len < 0 || q0 < 0 || k0 < 0 || q0 + q_len > a.M ||
+                     k0 + k_len > a.N || (mb == a.num_mblocks - 1 &&
+                                          q_len > a.num_mblocks * kFwdRowsPerCta);
+    if (bad) {
+      if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
+      return;
+    }
+  }
+  const int m_base = mb * kFwdRowsPerCta;
+  if (m_base >= q_len) return;
+  const int off = k_len - q_len;  // bottom-right causal alignment
+
+  // Key tiles each query tile needs.
+  int nt_tile[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int mt = m_base + t * kBM;
+    int nkeys = 0;
+    if (mt < q_len) {
+      nkeys = k_len;
+      if (kCausal) nkeys = min(k_len, max(0, mt + kBM + off));
+    }
+    nt_tile[t] = (nkeys + kBN - 1) / kBN;
+  }
+  const int nt = max(nt_tile[0], nt_tile[1]);
+
+  // ---- set-up -----------------------------------------------------------
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_ready[t], kBM);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ===================== TMA producer =====================================
+    if (lane == 0 && nt > 0) {
+      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, q_full, c * 64, h,
+                      q0 + m_base + t * kBM, bidx);
+      int it = 0;
+      for (int j = 0; j < nt; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int slot = it % S;
+          if (!mbar_wait(&kv_empty[slot], ((it / S) & 1) ^ 1, abort_flag, a.status)) break;
+          mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+          const CUtensorMap* map = kv ? &tmV : &tmK;
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
+                        c * 64, kvh, k0 + j * kBN, bidx);
+        }
+        if (*abort_flag) break;
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      mbar_wait_drain(q_full, 0, a.status);
+      for (int i = max(0, it - S); i < it; ++i)
+        mbar_wait_drain(&kv_full[i % S], (i / S) & 1, a.status);
+    }
+  } else if (warp == kMmaWarp) {
+    // ===================== MMA issuer =======================================
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_f16(BF16, kBM, kBN, false);
+      const uint32_t idesc_pv = idesc_f16(BF16, kBM, D, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t kv_addr = smem_u32(sKV);
+      // S_t = Q_t K^T: both operands K-major; step k advances 16 elements (32 bytes)
+      // inside a 128-byte swizzle row, then to the next 64-column chunk.
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t d = tmem_base + t * kBN;
+        const uint32_t qa = q_addr + t * L::kTileBytes;
+        const uint32_t kb = kv_addr + slot * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+          umma_ss(d, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(kb + o, 16, 1024), idesc_qk,
+                  kk > 0);
+        }
+      };
+      // O_t (+)= P_t V: P from TMEM (2 elements per column), V N-major with its
+      // 64-column chunks L::kChunkBytes apart; step k covers 16 keys = 2048 bytes.
+      auto issue_pv = [&](int t, int slot, bool accumulate) {
+        const uint32_t d = tmem_base + 2 * kBN + t * D;
+        const uint32_t p = tmem_base + t * kBN;
+        const uint32_t vb = kv_addr + slot * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts(d, p + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
+                  (accumulate || kk > 0) ? 1u : 0u);
+      };
+
+      if (nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
+        int it = 0, vslot_prev = 0;
+        bool ok = true;
+        for (int j = 0; j < nt && ok; ++j) {
+          const int kslot = it % S;
+          if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
+          ++it;
+          tc_fence_after();
+          if (j < nt_tile[0]) {
+            issue_qk(0, kslot);
+            umma_commit(&s_full[0]);
+          }
+          if (j >= 1) {
+            if (j - 1 < nt_tile[1]) {
+              if (!(ok = mbar_wait(&p_ready[1], (j - 1) & 1, abort_flag, a.status))) break;
+              tc_fence_after();
+              issue_pv(1, vslot_prev, j - 1 > 0);
+              umma_commit(&o_done[1]);
+            }
+            umma_commit(&kv_empty[vslot_prev]);
+          }
+          if (j < nt_tile[1]) {
+            issue_qk(1, kslot);
+            umma_commit(&s_full[1]);
+          }
+          umma_commit(&kv_empty[kslot]);
+          const int vslot = it % S;
+          if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
+          ++it;
+          tc_fence_after();
+          if (j < nt_tile[0]) {
+            if (!(ok = mbar_wait(&p_ready[0], j & 1, abort_flag, a.status))) break;
+            tc_fence_after();
+            issue_pv(0, vslot, j > 0);
+            umma_commit(&o_done[0]);
+          }
+          vslot_prev = vslot;
+        }
+        if (ok) {
+          const int j = nt - 1;
+          if (j < nt_tile[1] && mbar_wait(&p_ready[1], j & 1, abort_flag, a.status)) {
+            tc_fence_after();
+            issue_pv(1, vslot_prev, j > 0);
+            umma_commit(&o_done[1]);
+          }
+          umma_commit(&kv_empty[vslot_prev]);
+        }
+      }
+      // Every MMA issued above has completed once this barrier flips.
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0, a.status);
+    }
+  } else {
+    // ===================== softmax warpgroups ===============================
+    const int t = warp >> 2;                   // query tile
+    const int wq = warp & 3;                   // TMEM lane quarter
+    const int row = wq * 32 + lane;            // row inside the tile
+    const int r = m_base + t * kBM + row;      // row inside the sequence
+    const int pos_i = r + off;                 // its position in key coordinates
+    const int ntt = nt_tile[t];
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_addr = tmem_base + lane_addr + t * kBN;
+    const uint32_t o_addr = tmem_base + lane_addr + 2 * kBN + t * D;
+    float slope_log2 = 0.f;
+    if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
+
+    float m_ref = neg_inf();  // reference max (log2 units) used for the exponentials
+    float l_sum = 0.f;        // running sum of 2^(x - m_ref)
+    bool ok = true;
+
+    for (int j = 0; j < ntt; ++j) {
+      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+
+      // scale (+ ALiBi), mask, row max -- all in log2 units
+      const int n0 = j * kBN;
+      int limit = k_len - n0;
+      if (kCausal) limit = min(limit, pos_i + 1 - n0);
+      const bool full = limit >= kBN;
+      float mx = neg_inf();
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        float x = __uint_as_float(sr[c >> 5][c & 31]) * a.scale_log2;
+        if constexpr (ALIBI)
+          x = fmaf(-slope_log2, fabsf(static_cast<float>(n0 + c - pos_i)), x);
+        if (!full && c >= limit) x = neg_inf();
+        sr[c >> 5][c & 31] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      float m_use = m_ref;
+      if (mx > m_ref + kTau) m_use = mx;  // also taken when m_ref is -inf
+      const float alpha = (m_use == m_ref) ? 1.f : ex2(m_ref - m_use);
+      m_ref = m_use;
+      const float m_sub = (m_use == neg_inf()) ? 0.f : m_use;
+
+      // P = 2^(x - m), row sum, pack to 16-bit pairs and store over S
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(__uint_as_float(sr[c][2 * i]) - m_sub);
+          const float p1 = ex2(__uint_as_float(sr[c][2 * i + 1]) - m_sub);
+          sum0 += p0;
+          sum1 += p1;
+          pk[i] = pack2<BF16>(p0, p1);
+        }
+        tmem_st16(s_addr + c * 16, pk);
+      }
+      l_sum = l_sum * alpha + (sum0 + sum1);
+
+      // Rescale the output accumulator when this row's reference max moved.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!(ok = mbar_wait_warp(&o_done[t], (j - 1) & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(o_addr + c * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[t]);
+    }
+
+    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 -------------------
+    if (ok && ntt > 0) ok = mbar_wait_warp(&o_done[t], (ntt - 1) & 1, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = r < q_len;
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
+                      2 * (bidx * a.o_sb + static_cast<long long>(q0 + r) * a.o_sm + h * a.o_sh);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (ntt > 0) {
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
+                              __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (valid && a.lse != nullptr) {
+        const float lse = l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : neg_inf();
+        a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + r] = lse;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int D, bool BF16, int MASK, bool ALIBI>
+cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
+  auto kern = fwd_kernel<D, BF16, MASK, ALIBI>;
+  const int smem = Smem<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = static_cast<long long>(L.args.num_mblocks) * L.args.Hq *
+                         L.args.num_units;
+  if (grid <= 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.args);
+  return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+cudaError_t dispatch_mask(const FwdLaunch& L, cudaStream_t s) {
+  switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
+    case 0: return launch_t<D, BF16, 0, false>(L, s);
+    case 1: return launch_t<D, BF16, 0, true>(L, s);
+    case 2: return launch_t<D, BF16, 1, false>(L, s);
+    case 3: return launch_t<D, BF16, 1, true>(L, s);
+    case 4: return launch_t<D, BF16, 2, false>(L, s);
+    case 5: return launch_t<D, BF16, 2, true>(L, s);
+    case 6: return launch_t<D, BF16, 3, false>(L, s);
+    case 7: return launch_t<D, BF16, 3, true>(L, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+__global__ void fill_empty_kernel(uint16_t* out, float* lse, int B, int M, int Hq, int K,
+                                  long long o_sb, long long o_sm, long long o_sh) {
+  const long long rows = static_cast<long long>(B) * M * Hq;
+  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; r < rows;
+       r += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long b = r / (static_cast<long long>(M) * Hq);
+    const long long i = (r / Hq) % M;
+    const long long h = r % Hq;
+    uint16_t* row = out + b * o_sb + i * o_sm + h * o_sh;
+    for (int d = 0; d < K; ++d) row[d] = 0;
+    if (lse) lse[(b * Hq + h) * M + i] = neg_inf();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdLaunch& L, cudaStream_t stream) {
+  if (L.head_dim == 64)
+    return L.bf16 ? dispatch_mask<64, true>(L, stream) : dispatch_mask<64, false>(L, stream);
+  if (L.head_dim == 128)
+    return L.bf16 ? dispatch_mask<128, true>(L, stream) : dispatch_mask<128, false>(L, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fill_empty(void* out, float* lse, int B, int M, int Hq, int K, long long o_sb,
+                              long long o_sm, long long o_sh, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * M * Hq;
+  if (rows <= 0) return cudaSuccess;
+  const int threads = 256;
+  const long long blocks = min((rows + threads - 1) / threads, 4096LL);
+  fill_empty_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      static_cast<uint16_t*>(out), lse, B, M, Hq, K, o_sb, o_sm, o_sh);
+  return cudaGetLastError();
+}
+
+}  // namespace mea

@@ -1,0 +1,67 @@
+// mea_internal.h -- launch descriptions shared between the C-ABI translation unit
+// and the kernel translation units (host side only; no kernel code here).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <stdint.h>
+
+namespace mea {
+
+// Prefill: one CTA computes two 128-row query tiles of one (sequence, head).
+constexpr int kFwdRowsPerCta = 256;
+
+struct FwdArgs {
+  void* out;
+  float* lse;                  // [B, Hq, M] or nullptr
+  const int32_t* seqstart_q;   // packed batches only
+  const int32_t* seqstart_k;
+  int* status;                 // device status word
+  long long o_sb, o_sm, o_sh;  // out strides (elements)
+  int B, M, N, Hq, Hkv, group;
+  int num_units;    // B for dense batches, num_seqs for packed ones
+  int num_mblocks;  // ceil(max query rows per unit / kFwdRowsPerCta)
+  float scale_log2; // scale * log2(e)
+};
+
+struct FwdLaunch {
+  CUtensorMap tmQ, tmK, tmV;
+  FwdArgs args;
+  int head_dim;   // 64 or 128
+  bool bf16;
+  int mask;       // mea_bias_t value
+  bool alibi;
+};
+
+cudaError_t launch_fwd(const FwdLaunch& launch, cudaStream_t stream);
+
+// Rows with no visible key (or an empty key set): out = 0, lse = -inf.
+cudaError_t launch_fill_empty(void* out, float* lse, int B, int M, int Hq, int K, long long o_sb,
+                              long long o_sm, long long o_sh, cudaStream_t stream);
+
+// Decode: split-KV partial kernel + log-sum-exp merge.
+constexpr int kDecodeChunk = 512;  // cache rows per split
+
+struct DecodeArgs {
+  const void* q;               // [B, Hq, K]
+  void* out;                   // [B, Hq, K]
+  float* lse;                  // [B, Hq] or nullptr
+  const int32_t* kv_seqstart;  // [B + 1]
+  float* part_o;               // [B, Hq, max_splits, K]
+  float* part_lse;             // [B, Hq, max_splits] (log2 domain)
+  int* status;
+  int B, Hq, Hkv, group, max_splits, cache_rows;
+  float scale_log2;
+};
+
+struct DecodeLaunch {
+  CUtensorMap tmK, tmV;
+  DecodeArgs args;
+  int head_dim;
+  bool bf16;
+  bool alibi;
+};
+
+cudaError_t launch_decode(const DecodeLaunch& launch, cudaStream_t stream);
+
+}  // namespace mea
