@@ -459,12 +459,14 @@ def run_reference(args, rank, world):
     per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(p, per_step / 4)
+    t_start = time.perf_counter()
     vals = [cpu_baseline(p, per_step) for _ in range(args.steps)]
+    ms_per_step = (time.perf_counter() - t_start) * 1e3 / max(1, args.steps)
     v = statistics.mean(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = round(v, 6)
     return {"metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": 8, "H": 16, "K": 64,
@@ -474,19 +476,61 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+PROFILE_CASES = {
+    # small cases for ncu captures: inputs larger than L2, a few hundred MB at most
+    "fwd_sweep_m2048": lambda: ("fwd", synth.noncausal_sweep(2048)),
+    "fwd_gqa_alibi_m2048": lambda: ("fwd", synth.gqa_alibi_causal(M=2048, B=2)),
+    "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
+    "decode_b16": lambda: ("decode", synth.make_decode(
+        "decode_b16", synth.decode_lengths()[:16], 32, 8, 128, "bf16", seed=1005)),
+}
+
+
+def run_profile(args):
+    """Launch one workload W + K times (no JSON): the target of an ncu capture."""
+    import memory_efficient_exact_mea_b200 as mea
+
+    kind, w = PROFILE_CASES[args.profile]()
+    dev = torch.device("cuda", 0)
+    if kind == "fwd":
+        q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+        kw = {}
+        if w.seq_lens_q is not None:
+            kw = dict(seqstart_q=w.seqstart_q.to(dev), seqstart_k=w.seqstart_k.to(dev))
+
+        def fn():
+            mea.mea_fwd(q, k, v, bias=w.bias, scale=w.scale, alibi=w.alibi, **kw)
+    else:
+        q, kc, vc = w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev)
+        st = w.kv_seqstart.to(dev)
+
+        def fn():
+            mea.mea_decode(q, kc, vc, st, w.max_kv_len, scale=w.scale)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    assert mea.read_device_status() == 0
+    print(f"profiled {args.profile}: {args.warmup} + {args.steps} launches", flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="headline only, skip other workloads")
     ap.add_argument("--no-memory", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", choices=sorted(PROFILE_CASES),
+                    help="launch one small workload only (target for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.profile:
+        run_profile(args)
+        return
     rank, world, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":

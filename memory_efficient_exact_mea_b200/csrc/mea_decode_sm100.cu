@@ -236,8 +236,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         acc[mt][3] *= alpha[1];
       }
       // P^T as the B operand: transpose the (rows x heads) accumulator fragments.
-      const uint32_t pb0 = movmatrix_trans(pack2<BF16>(p[0], p[1]));
-      const uint32_t pb1 = movmatrix_trans(pack2<BF16>(p[2], p[3]));
+      // bf16 keeps only 8 significant bits, so P goes in as P_hi + P_lo.
+      const uint32_t ph0 = pack2<BF16>(p[0], p[1]);
+      const uint32_t ph1 = pack2<BF16>(p[2], p[3]);
+      const uint32_t pb0 = movmatrix_trans(ph0);
+      const uint32_t pb1 = movmatrix_trans(ph1);
+      uint32_t pl0 = 0u, pl1 = 0u;
+      if constexpr (BF16) {
+        pl0 = movmatrix_trans(pack2<BF16>(p[0] - __uint_as_float(ph0 << 16),
+                                          p[1] - __uint_as_float(ph0 & 0xffff0000u)));
+        pl1 = movmatrix_trans(pack2<BF16>(p[2] - __uint_as_float(ph1 << 16),
+                                          p[3] - __uint_as_float(ph1 & 0xffff0000u)));
+      }
       // O^T (dims x heads) += V^T . P^T
       {
         const int mi = lane >> 3, rr = lane & 7;
@@ -247,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t af[4];
           ldsm_x4_trans(vt + swz<D>(row, 2 * mt + (mi & 1)), af);
           mma16816<BF16>(acc[mt], af, pb0, pb1);
+          if constexpr (BF16) mma16816<BF16>(acc[mt], af, pl0, pl1);
         }
       }
       __syncwarp();

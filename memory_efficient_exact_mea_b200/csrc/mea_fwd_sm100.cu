@@ -15,9 +15,10 @@
 //   warp  8    TMEM allocator and the single MMA-issuing thread
 //   warp  9    the single TMA-issuing thread
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
-// current key tile; P = exp(S - m) in fp16/bf16 is written back over the first
-// 64 columns and fed to the P.V MMA straight from TMEM) | O0 | O1 (K columns
-// each, the fp32 output accumulators).
+// current key tile; P = exp(S - m) in fp16 is written back over the first 64
+// columns, in bf16 as P_hi over the first 64 and P_lo = P - P_hi over the last
+// 64, and fed to the P.V MMA straight from TMEM) | O0 | O1 (K columns each, the
+// fp32 output accumulators).
 // Shared memory: Q0, Q1 (loaded once) and a ring of key/value tiles, all in the
 // 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = Smem<D>;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
+  constexpr bool kSplitP = BF16;  // P.V as (P_hi + P_lo).V for bf16
   constexpr int S = L::kSlots;
 
   extern __shared__ uint8_t smem_raw[];
@@ -203,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_t (+)= P_t V: P from TMEM (2 elements per column), V N-major with its
       // 64-column chunks L::kChunkBytes apart; step k covers 16 keys = 2048 bytes.
+      // With the bf16 split, the low part P_lo (columns 64..127) goes through
+      // the same V descriptors.
       auto issue_pv = [&](int t, int slot, bool accumulate) {
         const uint32_t d = tmem_base + 2 * kBN + t * D;
         const uint32_t p = tmem_base + t * kBN;
@@ -211,6 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBN / 16; ++kk)
           umma_ts(d, p + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
                   (accumulate || kk > 0) ? 1u : 0u);
+        if constexpr (kSplitP) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ts(d, p + kBN / 2 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024),
+                    idesc_pv, 1u);
+        }
       };
 
       if (nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
@@ -313,11 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_ref = m_use;
       const float m_sub = (m_use == neg_inf()) ? 0.f : m_use;
 
-      // P = 2^(x - m), row sum, pack to 16-bit pairs and store over S
+      // P = 2^(x - m), row sum, pack to 16-bit pairs and store over S.  With
+      // bf16 (8 significant bits) P is stored as hi + lo, two bf16 matrices in
+      // columns [0, 64) and [64, 128), so that P.V carries ~16 bits of P.
       float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t pk[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2(__uint_as_float(sr[c][2 * i]) - m_sub);
@@ -325,8 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum0 += p0;
           sum1 += p1;
           pk[i] = pack2<BF16>(p0, p1);
+          if constexpr (kSplitP)
+            lo[i] = pack2<BF16>(p0 - __uint_as_float(pk[i] << 16),
+                                p1 - __uint_as_float(pk[i] & 0xffff0000u));
         }
         tmem_st16(s_addr + c * 16, pk);
+        if constexpr (kSplitP) tmem_st16(s_addr + kBN / 2 + c * 16, lo);
       }
       l_sum = l_sum * alpha + (sum0 + sum1);
 
