@@ -143,6 +143,41 @@ int mea_decode(const void* q, const void* k_cache, const void* v_cache,
                mea_dtype_t dtype, int alibi, float scale,
                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * mea_decode_noalloc -- mea_decode without a caller-provided workspace.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory at the point of the call.  Examples: a plugin
+ * or plain C host program embedded in a runtime that owns all device memory
+ * through its own pool and hands it no allocator, or a serving loop that must
+ * not call cudaMalloc after start-up, because cudaMalloc can synchronise the
+ * device and can fail once memory is exhausted.
+ *
+ * Arguments, layouts and results are those of mea_decode.  The split partials
+ * go to a fixed 32 MiB device array inside this library instead of a workspace,
+ * which bounds the problem size to
+ *     mea_decode_workspace_size(B, Hq, Hkv, K, max_kv_len) <= 32 MiB
+ * (e.g. B=64, Hq=32, K=128, max_kv_len=8192 needs 16.9 MB).  Larger problems
+ * return MEA_ERR_WORKSPACE before anything is launched.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree and no allocating library routine.
+ *
+ * Notes for callers:
+ *  - Every GPU that loads this library holds the 32 MiB array until the
+ *    process exits.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current, and caches it.  Make that first call before any stream
+ *    capture begins.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents.  Nothing in it has to start at zero: every partial a call reads,
+ *    the same call has written first.  Calls whose executions overlap on the GPU
+ *    (different streams, or different host threads) race on the array and give
+ *    wrong results; serialise them.
+ */
+int mea_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* kv_seqstart, void* out, float* lse,
+                       int B, int Hq, int Hkv, int K, int cache_rows, int max_kv_len,
+                       mea_dtype_t dtype, int alibi, float scale, cudaStream_t stream);
+
 /* Number of key/value rows one decode split covers (the unit of parallelism). */
 int mea_decode_chunk(void);
 

@@ -19,6 +19,9 @@
 //   * a second kernel merges the chunk partials exactly by their log-sum-exp.
 #include <math.h>
 
+#include <mutex>
+
+#include "mea.h"
 #include "mea_internal.h"
 #include "sm100.cuh"
 
@@ -386,6 +389,41 @@ cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t stream) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode: the split partials live in a fixed device array that
+// belongs to this library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
+constexpr int kMaxDevices = 64;
+
+// Every device that loads this library holds this array until the process exits.
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_decode_scratch on the current device.  Host code cannot use
+// the symbol itself (on the host it names a stand-in, not device memory), so the
+// address is looked up once per device, with that device current, and cached.
+cudaError_t noalloc_scratch(void** ptr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  static std::mutex mu;
+  static void* cached[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = p;
+  }
+  *ptr = cached[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
   const int key = (L.head_dim == 128 ? 4 : 0) + (L.bf16 ? 2 : 0) + (L.alibi ? 1 : 0);
   if (L.head_dim != 64 && L.head_dim != 128) return cudaErrorInvalidValue;
@@ -403,3 +441,19 @@ cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t stream) {
 }
 
 }  // namespace mea
+
+// The allocation-free entry point (declared in mea.h).  It validates the size
+// against the built-in scratch and then runs exactly the mea_decode path with
+// that scratch as its workspace.
+extern "C" int mea_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* kv_seqstart, void* out, float* lse, int B,
+                                  int Hq, int Hkv, int K, int cache_rows, int max_kv_len,
+                                  mea_dtype_t dtype, int alibi, float scale,
+                                  cudaStream_t stream) {
+  const size_t need = mea_decode_workspace_size(B, Hq, Hkv, K, max_kv_len);
+  if (need > mea::kNoAllocScratchBytes) return MEA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (mea::noalloc_scratch(&scratch) != cudaSuccess) return MEA_ERR_CUDA;
+  return mea_decode(q, k_cache, v_cache, kv_seqstart, out, lse, B, Hq, Hkv, K, cache_rows,
+                    max_kv_len, dtype, alibi, scale, scratch, mea::kNoAllocScratchBytes, stream);
+}
