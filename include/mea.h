@@ -96,7 +96,8 @@ typedef enum {
  * alibi:  nonzero adds -slope_h * |pos_i - pos_j| after scaling, positions local
  *         to the sequence with pos_i = i + (N - M), slope_h = 2^(-8 (h+1) / Hq)
  *         computed in registers (tutorial section "Utilizzare SwiGLU e ALiBi").
- * scale:  multiplies q.k (pass 1/sqrt(K) for the usual attention).
+ * scale:  multiplies q.k (pass 1/sqrt(K) for the usual attention); must be >= 0
+ *         (a negative scale returns MEA_ERR_UNSUPPORTED: negate q instead).
  *
  * A query row that sees no key gets out = 0 and lse = -inf.
  * Returns MEA_OK or an error status; never synchronises.

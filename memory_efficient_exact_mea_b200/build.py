@@ -19,33 +19,35 @@ FLAGS = [
 ]
 
 
-def build(verbose: bool = False, jobs: int = 3) -> str:
+def build(verbose: bool = False, extra_flags=(), out: str | None = None,
+          build_dir: str | None = None) -> str:
     """Compile every translation unit (in parallel) and link libmea.so."""
-    build_dir = os.path.join(ROOT, "_build")
+    build_dir = build_dir or os.path.join(ROOT, "_build")
     os.makedirs(build_dir, exist_ok=True)
     inc = ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
     procs, objs = [], []
     for src in SOURCES:
         obj = os.path.join(build_dir, src.replace(".cu", ".o"))
         objs.append(obj)
-        cmd = [NVCC, *FLAGS, *inc, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [NVCC, *FLAGS, *extra_flags, *inc, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE,
                                             stderr=subprocess.STDOUT, text=True)))
     failed = []
     for src, p in procs:
-        out, _ = p.communicate()
+        log, _ = p.communicate()
         if verbose or p.returncode:
-            sys.stderr.write(out)
+            sys.stderr.write(log)
         if p.returncode:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for {failed}")
-    tmp = LIB + f".tmp{os.getpid()}"
+    out = out or LIB
+    tmp = out + f".tmp{os.getpid()}"
     subprocess.run([NVCC, *FLAGS, *objs, "-o", tmp], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -123,6 +123,7 @@ int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   if (B == 0 || M == 0) return MEA_OK;
   if (!q || !out || (N > 0 && (!k || !v))) return MEA_ERR_INVALID_ARG;
   if (K != 64 && K != 128) return MEA_ERR_UNSUPPORTED;
+  if (scale < 0.f) return MEA_ERR_UNSUPPORTED;  // the kernel takes row maxima on raw scores
   const bool packed = bias == MEA_BIAS_BLOCKDIAG || bias == MEA_BIAS_BLOCKDIAG_CAUSAL;
   if (packed) {
     if (B != 1 || !seqstart_q || num_seqs <= 0 || max_seqlen_q < 0) return MEA_ERR_INVALID_ARG;

@@ -9,16 +9,18 @@
 // Transformer efficienti in memoria con xFormers ...", "Applicare Attenzione
 // Causale con Maschere Inferiori", "Utilizzare Sequenze di Lunghezza Variabile").
 //
-// CTA organisation (320 threads, one CTA per SM):
-//   warps 0-3  softmax / rescale / epilogue for query tile 0 (TMEM lanes 0-127)
-//   warps 4-7  the same for query tile 1 (rows +128)
-//   warp  8    TMEM allocator and the single MMA-issuing thread
-//   warp  9    the single TMA-issuing thread
+// CTA organisation (576 threads, one CTA per SM):
+//   warps 0-7   softmax / rescale / epilogue for query tile 0 (TMEM lanes 0-127):
+//               two threads per row, warps 0-3 on score columns 0-63 and the
+//               first half of the output row, warps 4-7 on the other halves
+//   warps 8-15  the same for query tile 1 (rows +128)
+//   warp  16    TMEM allocator and the single MMA-issuing thread
+//   warp  17    the single TMA-issuing thread
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
-// current key tile; P = exp(S - m) in fp16 is written back over the first 64
-// columns, in bf16 as P_hi over the first 64 and P_lo = P - P_hi over the last
-// 64, and fed to the P.V MMA straight from TMEM) | O0 | O1 (K columns each, the
-// fp32 output accumulators).
+// current key tile; P = exp(S - m) as 16-bit pairs is written back over S, each
+// 32-key chunk over its own 32 columns: fp16 P in the first 16, bf16 as P_hi in
+// the first 16 and P_lo = P - P_hi in the last 16; the P.V MMA reads P straight
+// from TMEM) | O0 | O1 (K columns each, the fp32 output accumulators).
 // Shared memory: Q0, Q1 (loaded once) and a ring of key/value tiles, all in the
 // 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
@@ -31,9 +33,10 @@ namespace {
 
 constexpr int kBM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;        // keys per tile
-constexpr int kThreads = 320;
-constexpr int kMmaWarp = 8;
-constexpr int kTmaWarp = 9;
+constexpr int kThreads = 576;
+constexpr int kMmaWarp = 16;
+constexpr int kTmaWarp = 17;
+constexpr int kSoftmaxThreadsPerTile = 256;  // two threads per row
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceeds it by < 2^8
 constexpr float kLog2e = 1.4426950408889634f;
@@ -48,13 +51,35 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kKV = 2 * kTileBytes;
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
-  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1 + 8 + 2;
+  // Row-pair exchange: partial maxima [tile][parity][half][row], sums [tile][half][row].
+  static constexpr int kXMax = kBar + kNumBars * 8;
+  static constexpr int kXSum = kXMax + 2 * 2 * 2 * kBM * 4;
+  static constexpr int kTmemSlot = kXSum + 2 * 2 * kBM * 4;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// Pipeline timeline for performance work: built only with -DMEA_TRACE, it
+// records clock64() at each pipeline event of the first kTraceCtas CTAs.
+// Slots per CTA: softmax tile t, key tile j, event e -> t*512 + j*16 + e;
+// MMA thread, key tile j, event e -> 1024 + j*16 + e (j < 32).
+#ifdef MEA_TRACE
+constexpr int kTraceCtas = 4;
+constexpr int kTraceSlots = 1536;
+__device__ long long g_trace[kTraceCtas * kTraceSlots];
+#define MEA_TRACE_AT(slot)                                                         \
+  do {                                                                             \
+    if (blockIdx.x < kTraceCtas && (slot) < kTraceSlots)                           \
+      g_trace[blockIdx.x * kTraceSlots + (slot)] = clock64();                      \
+  } while (0)
+#else
+#define MEA_TRACE_AT(slot) \
+  do {                     \
+  } while (0)
+#endif
 
 template <int D, bool BF16, int MASK, bool ALIBI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -64,6 +89,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
   constexpr bool kSplitP = BF16;  // P.V as (P_hi + P_lo).V for bf16
+  // With K = 64 and fp16, P gets TMEM columns of its own (S 2x128, P 2x64, O 2x64
+  // = 512), so S_t is free as soon as the softmax has read it and the next
+  // Q.K^T of the same tile runs during its softmax.  Otherwise P is written over S.
+  constexpr bool kSepP = (D == 64) && !BF16;
+  constexpr uint32_t kColP = kSepP ? 2 * kBN : 0;          // + t * (kSepP ? kBN/2 : kBN)
+  constexpr uint32_t kColO = kSepP ? 2 * kBN + kBN : 2 * kBN;  // + t * D
   constexpr int S = L::kSlots;
 
   extern __shared__ uint8_t smem_raw[];
@@ -79,6 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_ready = s_full + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* mma_done = o_done + 2;
+  uint64_t* pair_bar = mma_done + 1;  // [tile][lane quarter]: the two warps of a row pair
+  uint64_t* s_free = pair_bar + 8;    // S_t read out by the softmax (separate-P layout)
+  float* xmax = reinterpret_cast<float*>(smem + L::kXMax);
+  float* xsum = reinterpret_cast<float*>(smem + L::kXSum);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
@@ -136,10 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_ready[t], kBM);
+      mbar_init(&p_ready[t], kSoftmaxThreadsPerTile);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 64);
+    for (int t = 0; t < 2; ++t) mbar_init(&s_free[t], kSoftmaxThreadsPerTile);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -203,41 +240,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kk > 0);
         }
       };
-      // O_t (+)= P_t V: P from TMEM (2 elements per column), V N-major with its
-      // 64-column chunks L::kChunkBytes apart; step k covers 16 keys = 2048 bytes.
-      // With the bf16 split, the low part P_lo (columns 64..127) goes through
-      // the same V descriptors.
+      // O_t (+)= P_t V: P from TMEM (2 elements per column; keys 32c..32c+31 in
+      // columns 32c..32c+15), V N-major with its 64-column chunks L::kChunkBytes
+      // apart; step k covers 16 keys = 2048 bytes of V.  With the bf16 split the
+      // low part P_lo (16 columns further) goes through the same V descriptors.
+      // Separate-P layout: keys 2c, 2c+1 in column c of P_t.
       auto issue_pv = [&](int t, int slot, bool accumulate) {
-        const uint32_t d = tmem_base + 2 * kBN + t * D;
-        const uint32_t p = tmem_base + t * kBN;
+        const uint32_t d = tmem_base + kColO + t * D;
+        const uint32_t p = tmem_base + kColP + t * (kSepP ? kBN / 2 : kBN);
         const uint32_t vb = kv_addr + slot * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(d, p + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
+          umma_ts(d, kSepP ? p + kk * 8 : p + (kk >> 1) * 32 + (kk & 1) * 8,
+                  sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
                   (accumulate || kk > 0) ? 1u : 0u);
         if constexpr (kSplitP) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts(d, p + kBN / 2 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024),
-                    idesc_pv, 1u);
+            umma_ts(d, p + (kk >> 1) * 32 + 16 + (kk & 1) * 8,
+                    sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv, 1u);
         }
       };
 
-      if (nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
+      if (kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
+        // Ring index 2j holds K_j, 2j+1 holds V_j.  Iteration j issues Q.K_j^T
+        // for both tiles (each once its S buffer has been read out), then P.V_{j-1}.
+        bool ok = true;
+        // Both tiles' MMAs go out as one batch (Q.K^T: 8 instructions, P.V: 16):
+        // every batch that starts after an idle tensor pipe pays its fill latency.
+        for (int j = 0; j <= nt && ok; ++j) {
+          if (j < nt) {
+            const int ks = (2 * j) % S;
+            if (!(ok = mbar_wait(&kv_full[ks], ((2 * j) / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + j * 16 + 0);
+            if (j > 0) {  // the softmax has read S_t out of TMEM
+              for (int t = 0; t < 2 && ok; ++t)
+                if (j < nt_tile[t]) ok = mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, a.status);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            MEA_TRACE_AT(1024 + j * 16 + 1);
+            for (int t = 0; t < 2; ++t) {
+              if (j >= nt_tile[t]) continue;
+              issue_qk(t, ks);
+              umma_commit(&s_full[t]);
+            }
+            MEA_TRACE_AT(1024 + j * 16 + 3);
+            umma_commit(&kv_empty[ks]);
+          }
+          if (j >= 1) {
+            const int jv = j - 1, vs = (2 * jv + 1) % S;
+            if (!(ok = mbar_wait(&kv_full[vs], ((2 * jv + 1) / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + j * 16 + 4);
+            for (int t = 0; t < 2 && ok; ++t)
+              if (jv < nt_tile[t]) ok = mbar_wait(&p_ready[t], jv & 1, abort_flag, a.status);
+            if (!ok) break;
+            MEA_TRACE_AT(1024 + j * 16 + 5);
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t) {
+              if (jv >= nt_tile[t]) continue;
+              issue_pv(t, vs, jv > 0);
+              umma_commit(&o_done[t]);
+            }
+            MEA_TRACE_AT(1024 + j * 16 + 6);
+            umma_commit(&kv_empty[vs]);
+          }
+        }
+      } else if (!kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
         int it = 0, vslot_prev = 0;
         bool ok = true;
         for (int j = 0; j < nt && ok; ++j) {
           const int kslot = it % S;
           if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
+          MEA_TRACE_AT(1024 + j * 16 + 0);
           ++it;
-          tc_fence_after();
           if (j < nt_tile[0]) {
             issue_qk(0, kslot);
+            MEA_TRACE_AT(1024 + j * 16 + 1);
             umma_commit(&s_full[0]);
           }
           if (j >= 1) {
             if (j - 1 < nt_tile[1]) {
               if (!(ok = mbar_wait(&p_ready[1], (j - 1) & 1, abort_flag, a.status))) break;
+              MEA_TRACE_AT(1024 + j * 16 + 2);
               tc_fence_after();
               issue_pv(1, vslot_prev, j - 1 > 0);
               umma_commit(&o_done[1]);
@@ -246,17 +331,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (j < nt_tile[1]) {
             issue_qk(1, kslot);
+            MEA_TRACE_AT(1024 + j * 16 + 3);
             umma_commit(&s_full[1]);
           }
           umma_commit(&kv_empty[kslot]);
           const int vslot = it % S;
           if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
+          MEA_TRACE_AT(1024 + j * 16 + 4);
           ++it;
-          tc_fence_after();
           if (j < nt_tile[0]) {
             if (!(ok = mbar_wait(&p_ready[0], j & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + j * 16 + 5);
             tc_fence_after();
             issue_pv(0, vslot, j > 0);
+            MEA_TRACE_AT(1024 + j * 16 + 6);
             umma_commit(&o_done[0]);
           }
           vslot_prev = vslot;
@@ -277,81 +365,150 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================== softmax warpgroups ===============================
-    const int t = warp >> 2;                   // query tile
+    // Two threads per row: `half` 0 owns score columns 0..63 of each key tile
+    // and output columns 0..D/2-1, `half` 1 the rest.  The two threads of a row
+    // (same lane in warps w and w+4) exchange partial row maxima every tile and
+    // partial row sums at the end through shared memory, ordered by an
+    // mbarrier of 64 arrivals (`pair_bar`), so both apply the same reference max.
+    const int t = warp >> 3;                   // query tile
+    const int half = (warp >> 2) & 1;          // column half
     const int wq = warp & 3;                   // TMEM lane quarter
     const int row = wq * 32 + lane;            // row inside the tile
     const int r = m_base + t * kBM + row;      // row inside the sequence
     const int pos_i = r + off;                 // its position in key coordinates
     const int ntt = nt_tile[t];
+    const int c0 = half * (kBN / 2);           // first score column of this thread
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t s_addr = tmem_base + lane_addr + t * kBN;
-    const uint32_t o_addr = tmem_base + lane_addr + 2 * kBN + t * D;
+    const uint32_t s_addr = tmem_base + lane_addr + t * kBN + c0;
+    const uint32_t o_addr = tmem_base + lane_addr + kColO + t * D + half * (D / 2);
+    // Where this thread's P goes: its own columns (separate-P layout, 16 packed
+    // columns per 32 keys) or over its S columns (32 per 32 keys, hi then lo).
+    const uint32_t p_addr = kSepP ? tmem_base + lane_addr + kColP + t * (kBN / 2) + half * (kBN / 4)
+                                  : s_addr;
+    uint64_t* pbar = &pair_bar[t * 4 + wq];
+    const bool tracer = (warp & 7) == 0 && lane == 0;
     float slope_log2 = 0.f;
     if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
 
     float m_ref = neg_inf();  // reference max (log2 units) used for the exponentials
-    float l_sum = 0.f;        // running sum of 2^(x - m_ref)
+    float l_sum = 0.f;        // this thread's part of the running sum of 2^(x - m_ref)
     bool ok = true;
 
     for (int j = 0; j < ntt; ++j) {
       if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag, a.status))) break;
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+      uint32_t sr[2][32];
+      tmem_ld32(s_addr, sr[0]);
+      tmem_ld32(s_addr + 32, sr[1]);
 
-      // scale (+ ALiBi), mask, row max -- all in log2 units
+      // Keys this row may see in the tile: columns [0, limit).  Tiles that need
+      // no masking for any row of the warp take the unmasked path (warp-uniform).
       const int n0 = j * kBN;
       int limit = k_len - n0;
       if (kCausal) limit = min(limit, pos_i + 1 - n0);
-      const bool full = limit >= kBN;
-      float mx = neg_inf();
-#pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        float x = __uint_as_float(sr[c >> 5][c & 31]) * a.scale_log2;
-        if constexpr (ALIBI)
-          x = fmaf(-slope_log2, fabsf(static_cast<float>(n0 + c - pos_i)), x);
-        if (!full && c >= limit) x = neg_inf();
-        sr[c >> 5][c & 31] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      const bool masked = __any_sync(0xffffffffu, limit < kBN);
+      const float dpos0 = static_cast<float>(n0 + c0 - pos_i);  // ALiBi distance of column c0
+      tmem_ld_wait(sr[0]);
+      tmem_ld_wait(sr[1]);
+      if constexpr (kSepP) {  // S_t may now be overwritten by the next Q.K^T
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);
       }
+
+      // ---- pass 1: partial row max (log2 units) ------------------------------
+      // Without ALiBi the max is taken on the raw scores (scale >= 0) and scaled
+      // once; with ALiBi the biased logit is formed here, in place.
+      float mx[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
+      if constexpr (ALIBI) {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i) {
+          float y = fmaf(__uint_as_float(sr[i >> 5][i & 31]), a.scale_log2,
+                         -slope_log2 * fabsf(dpos0 + static_cast<float>(i)));
+          if (masked && c0 + i >= limit) y = neg_inf();
+          sr[i >> 5][i & 31] = __float_as_uint(y);
+          mx[i & 3] = fmaxf(mx[i & 3], y);
+        }
+      } else if (!masked) {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; i += 2)
+          mx[(i >> 1) & 3] = max3(mx[(i >> 1) & 3], __uint_as_float(sr[i >> 5][i & 31]),
+                                  __uint_as_float(sr[i >> 5][(i + 1) & 31]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i)
+          if (c0 + i < limit) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i >> 5][i & 31]));
+      }
+      float pmax = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      if constexpr (!ALIBI) pmax = (pmax == neg_inf()) ? pmax : pmax * a.scale_log2;
+
+      // ---- exchange with the other half of the row -----------------------------
+      float* xm = xmax + ((t * 2 + (j & 1)) * 2) * kBM;
+      xm[half * kBM + row] = pmax;
+      mbar_arrive(pbar);
+      if (!(ok = mbar_wait_warp(pbar, j & 1, abort_flag, a.status))) break;
+      const float tmax = fmaxf(pmax, xm[(1 - half) * kBM + row]);
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
       float m_use = m_ref;
-      if (mx > m_ref + kTau) m_use = mx;  // also taken when m_ref is -inf
+      if (tmax > m_ref + kTau) m_use = tmax;  // also taken when m_ref is -inf
       const float alpha = (m_use == m_ref) ? 1.f : ex2(m_ref - m_use);
       m_ref = m_use;
-      const float m_sub = (m_use == neg_inf()) ? 0.f : m_use;
+      const float nsub = (m_use == neg_inf()) ? 0.f : -m_use;
 
-      // P = 2^(x - m), row sum, pack to 16-bit pairs and store over S.  With
-      // bf16 (8 significant bits) P is stored as hi + lo, two bf16 matrices in
-      // columns [0, 64) and [64, 128), so that P.V carries ~16 bits of P.
-      float sum0 = 0.f, sum1 = 0.f;
+      // ---- pass 2: P = 2^(logit - m) in place, partial row sums ----------------
+      f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
+      const f2 scale2 = {a.scale_log2, a.scale_log2}, nsub2 = {nsub, nsub};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int i = 0; i < kBN / 2; i += 2) {
+        const f2 v = {__uint_as_float(sr[i >> 5][i & 31]),
+                      __uint_as_float(sr[i >> 5][(i + 1) & 31])};
+        const f2 y = ALIBI ? add2(v, nsub2) : fma2(v, scale2, nsub2);
+        f2 p = {ex2(y.x), ex2(y.y)};
+        if (!ALIBI && masked) {
+          if (c0 + i >= limit) p.x = 0.f;
+          if (c0 + i + 1 >= limit) p.y = 0.f;
+        }
+        ps[(i >> 1) & 1] = add2(ps[(i >> 1) & 1], p);
+        sr[i >> 5][i & 31] = __float_as_uint(p.x);
+        sr[i >> 5][(i + 1) & 31] = __float_as_uint(p.y);
+      }
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+      if constexpr (kSepP) {  // P_t is still being read by P.V of the previous tile
+        if (j > 0 && !(ok = mbar_wait_warp(&o_done[t], (j - 1) & 1, abort_flag, a.status))) break;
+        tc_fence_after();
+      }
+      // Store P as 16-bit pairs over each 32-key chunk's own S columns (keys
+      // 32C..32C+31 -> columns 32C..32C+15).  With bf16 (8 significant bits) P
+      // is stored as hi + lo, the low part P - P_hi in columns 32C+16..32C+31,
+      // so that P.V carries ~16 bits of P.
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(__uint_as_float(sr[c][2 * i]) - m_sub);
-          const float p1 = ex2(__uint_as_float(sr[c][2 * i + 1]) - m_sub);
-          sum0 += p0;
-          sum1 += p1;
-          pk[i] = pack2<BF16>(p0, p1);
-          if constexpr (kSplitP)
-            lo[i] = pack2<BF16>(p0 - __uint_as_float(pk[i] << 16),
-                                p1 - __uint_as_float(pk[i] & 0xffff0000u));
+          const f2 p = {__uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1])};
+          pk[i] = pack2<BF16>(p.x, p.y);
+          if constexpr (kSplitP) {
+            const f2 hi = {__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u)};
+            const f2 res = fma2(hi, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
+            lo[i] = pack2<BF16>(res.x, res.y);
+          }
         }
-        tmem_st16(s_addr + c * 16, pk);
-        if constexpr (kSplitP) tmem_st16(s_addr + kBN / 2 + c * 16, lo);
+        tmem_st16(p_addr + c * (kSepP ? 16 : 32), pk);
+        if constexpr (kSplitP) tmem_st16(p_addr + c * 32 + 16, lo);
       }
-      l_sum = l_sum * alpha + (sum0 + sum1);
+      const f2 pst = add2(ps[0], ps[1]);
+      l_sum = l_sum * alpha + (pst.x + pst.y);
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
 
-      // Rescale the output accumulator when this row's reference max moved.
+      // Rescale this thread's half of the output accumulator when the row's
+      // reference max moved.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
         if (!(ok = mbar_wait_warp(&o_done[t], (j - 1) & 1, abort_flag, a.status))) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t o[32];
           tmem_ld32(o_addr + c * 32, o);
           tmem_ld_wait(o);
@@ -363,18 +520,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[t]);
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
     }
 
-    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 -------------------
+    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
     if (ok && ntt > 0) ok = mbar_wait_warp(&o_done[t], (ntt - 1) & 1, abort_flag, a.status);
     if (ok) {
+      // Row sum = both halves' parts (same reference max).
+      xsum[(t * 2 + half) * kBM + row] = l_sum;
+      mbar_arrive(pbar);
+      ok = mbar_wait_warp(pbar, ntt & 1, abort_flag, a.status);
+    }
+    if (ok) {
+      const float l_tot = l_sum + xsum[(t * 2 + 1 - half) * kBM + row];
       tc_fence_after();
       const bool valid = r < q_len;
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
-                      2 * (bidx * a.o_sb + static_cast<long long>(q0 + r) * a.o_sm + h * a.o_sh);
+                      2 * (bidx * a.o_sb + static_cast<long long>(q0 + r) * a.o_sm + h * a.o_sh +
+                           half * (D / 2));
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
         if (ntt > 0) {
           tmem_ld32(o_addr + c * 32, o);
@@ -395,8 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (valid && a.lse != nullptr) {
-        const float lse = l_sum > 0.f ? (m_ref + __log2f(l_sum)) * kLn2 : neg_inf();
+      if (valid && half == 0 && a.lse != nullptr) {
+        const float lse = l_tot > 0.f ? (m_ref + __log2f(l_tot)) * kLn2 : neg_inf();
         a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + r] = lse;
       }
     }
@@ -462,6 +628,14 @@ cudaError_t launch_fwd(const FwdLaunch& L, cudaStream_t stream) {
     return L.bf16 ? dispatch_mask<128, true>(L, stream) : dispatch_mask<128, false>(L, stream);
   return cudaErrorInvalidValue;
 }
+
+#ifdef MEA_TRACE
+// Copies the recorded timeline (kTraceCtas x kTraceSlots clock64 values) to host.
+extern "C" int mea_trace_read(long long* host, int n) {
+  if (n > kTraceCtas * kTraceSlots) n = kTraceCtas * kTraceSlots;
+  return cudaMemcpyFromSymbol(host, g_trace, n * sizeof(long long)) == cudaSuccess ? n : -1;
+}
+#endif
 
 cudaError_t launch_fill_empty(void* out, float* lse, int B, int M, int Hq, int K, long long o_sb,
                               long long o_sm, long long o_sh, cudaStream_t stream) {

@@ -93,6 +93,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert _fwd(lib, bias=3, sq=None, ns=1) == INVALID  # ... and offsets
     assert _fwd(lib, bias=2, sq=64, ns=1, N=9) == INVALID  # seqstart_k NULL needs M == N
     assert _fwd(lib, K=96) == UNSUPPORTED
+    assert _fwd(lib, scale=-0.5) == UNSUPPORTED
     assert _fwd(lib, q=24) == UNSUPPORTED               # 16-byte alignment
     assert _fwd(lib, qs=I64x3(1024, 100, 64)) == UNSUPPORTED  # stride not a multiple of 8
     assert _fwd(lib, qs=I64x3(1024, 128, 0)) == UNSUPPORTED
