@@ -278,13 +278,15 @@ def run_ours(args, rank, world, local):
         also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
     assert mea.read_device_status() == 0
 
-    traffic = traffic_for("fwd_kernel<64,f16,none>")
+    traffic = traffic_for("fwd_sweep")
     roofline = {
         "kernel": "fwd_kernel<K=64,f16,no mask> (sweep launches)",
         "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak,
         "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
         "peak_kind": f"{peaks_kind} bf16 burst (fp16 nominal rate = bf16)",
         "traffic": traffic,
+        "traffic_note": "mean DRAM read+write bytes per sweep launch (ncu, profiles/traffic.json);"
+                        " algorithmic q+k+v+out = 65536*M bytes, mean 125.8 MB",
         "algorithmic": "4*K*H*B*M*N FLOP per launch",
     }
     line = {
@@ -339,7 +341,9 @@ def memory_report(mea, p, q, k, v, dev):
 
 def measure_e2e(mea, sweep, dev, stream, args, world):
     """Same metric through the public call with host buffers: pinned H2D of q,k,v,
-    the kernel, D2H of out and lse, every step, inside the timed region."""
+    the kernel, D2H of out and lse, every step, inside the timed region.  Uploads,
+    kernels and downloads go on three streams, so the kernel of one sequence
+    length overlaps the upload of the next and the download of the previous."""
     host = [(p.q.pin_memory(), p.k.pin_memory(), p.v.pin_memory()) for p in sweep]
     dbuf = [(torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev),
              torch.empty_like(hv, device=dev)) for (hq, hk, hv) in host]
@@ -350,31 +354,51 @@ def measure_e2e(mea, sweep, dev, stream, args, world):
     h2d = sum(x.numel() * x.element_size() for t in host for x in t)
     d2h = sum(x.numel() * x.element_size() for x in houts) + sum(
         x.numel() * x.element_size() for x in hlses)
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = len(sweep)
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_kern = [torch.cuda.Event() for _ in range(n)]
+    ev_out = [torch.cuda.Event() for _ in range(n)]
+    first = [True]
 
     def step():
         for i, p in enumerate(sweep):
-            for dst, src in zip(dbuf[i], host[i]):
-                dst.copy_(src, non_blocking=True)
-            mea.mea_fwd(*dbuf[i], scale=p.scale, out=dout[i], lse=dlse[i])
-            houts[i].copy_(dout[i], non_blocking=True)
-            hlses[i].copy_(dlse[i], non_blocking=True)
+            if not first[0]:
+                s_up.wait_event(ev_kern[i])      # inputs i consumed by the previous step
+                stream.wait_event(ev_out[i])     # outputs i downloaded by the previous step
+            with torch.cuda.stream(s_up):
+                for dst, src in zip(dbuf[i], host[i]):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[i].record(s_up)
+            stream.wait_event(ev_in[i])
+            mea.mea_fwd(*dbuf[i], scale=p.scale, out=dout[i], lse=dlse[i], stream=stream)
+            ev_kern[i].record(stream)
+            s_down.wait_event(ev_kern[i])
+            with torch.cuda.stream(s_down):
+                houts[i].copy_(dout[i], non_blocking=True)
+                hlses[i].copy_(dlse[i], non_blocking=True)
+                ev_out[i].record(s_down)
+        first[0] = False
 
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
-    n = max(1, min(args.steps, 5))
+    n_steps = max(1, min(args.steps, 10))
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n):
+    e0.record(s_up)
+    for _ in range(n_steps):
         step()
-    e1.record(stream)
+    s_up.wait_stream(s_down)
+    s_up.wait_stream(stream)
+    e1.record(s_up)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    flops = sum(prefill_flops(p) for p in sweep) * n * world
+    flops = sum(prefill_flops(p) for p in sweep) * n_steps * world
     return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
-            "ms_per_step": round(ms / n, 3)}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_steps,
+            "ms_per_step": round(ms / n_steps, 3),
+            "overlap": "uploads, kernels and downloads on three streams"}
 
 
 def _time(fn, stream, iters, warmup=3):
@@ -478,6 +502,7 @@ def run_reference(args, rank, world):
 
 PROFILE_CASES = {
     # small cases for ncu captures: inputs larger than L2, a few hundred MB at most
+    "fwd_sweep_all": lambda: ("sweep", None),
     "fwd_sweep_m2048": lambda: ("fwd", synth.noncausal_sweep(2048)),
     "fwd_gqa_alibi_m2048": lambda: ("fwd", synth.gqa_alibi_causal(M=2048, B=2)),
     "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
@@ -492,7 +517,14 @@ def run_profile(args):
 
     kind, w = PROFILE_CASES[args.profile]()
     dev = torch.device("cuda", 0)
-    if kind == "fwd":
+    if kind == "sweep":  # one launch per sweep size per step
+        sweep = [synth.noncausal_sweep(M) for M in synth.SWEEP_M]
+        ins = [(p.q.to(dev), p.k.to(dev), p.v.to(dev), p.scale) for p in sweep]
+
+        def fn():
+            for q, k, v, sc in ins:
+                mea.mea_fwd(q, k, v, scale=sc)
+    elif kind == "fwd":
         q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
         kw = {}
         if w.seq_lens_q is not None:

@@ -192,6 +192,16 @@ const char* mea_status_string(int status);
  */
 int mea_read_device_status(cudaStream_t stream, int clear);
 
+/*
+ * mea_selftest_timeout -- exercises the failure path of the bounded waits.
+ * Launches one CTA that waits, through the same bounded mbarrier wait the
+ * kernels use, on a barrier nothing arrives on, and gives up after timeout_us
+ * microseconds (1 .. 10^7, else MEA_ERR_INVALID_ARG).  Afterwards the device
+ * status word holds MEA_ERR_DEVICE_TIMEOUT (see mea_read_device_status) and the
+ * CUDA context stays usable: nothing faults, traps or hangs.
+ */
+int mea_selftest_timeout(int timeout_us, cudaStream_t stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mea_version(void);
 

@@ -8,6 +8,7 @@
 
 #include "mea.h"
 #include "mea_internal.h"
+#include "sm100.cuh"
 
 // First error recorded by a kernel of this library (one word per device).
 __device__ int g_mea_status = 0;
@@ -252,3 +253,31 @@ int mea_read_device_status(cudaStream_t stream, int clear) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Failure-path self-test: one CTA waits on an mbarrier that nothing will ever
+// arrive on, through the same bounded wait the kernels use, with a short limit.
+// ---------------------------------------------------------------------------
+namespace {
+
+__global__ void selftest_timeout_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mea::mbar_init(&bar, 1);
+    abort_flag = 0;
+    mea::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mea::mbar_wait(&bar, 0, &abort_flag, status, timeout_ns);
+}
+
+}  // namespace
+
+extern "C" int mea_selftest_timeout(int timeout_us, cudaStream_t stream) {
+  if (timeout_us <= 0 || timeout_us > 10000000) return MEA_ERR_INVALID_ARG;
+  int* status = status_word();
+  if (!status) return MEA_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, 1000ull * timeout_us);
+  return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}

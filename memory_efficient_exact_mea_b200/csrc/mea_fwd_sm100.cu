@@ -121,12 +121,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- which (query block, head, batch or sequence) this CTA owns ----------
-  const int per_mb = a.Hq * a.num_units;
-  int mb = blockIdx.x / per_mb;
-  const int rem = blockIdx.x - mb * per_mb;
+  // The query block varies fastest, so the blocks of one (head, batch) -- and
+  // the heads sharing a key/value head -- run together and read each K/V tile
+  // from L2 instead of DRAM.  Under a causal mask the longest rows go first.
+  int mb = blockIdx.x % a.num_mblocks;
+  const int rem = blockIdx.x / a.num_mblocks;
   const int h = rem % a.Hq;
   const int unit = rem / a.Hq;
-  if (kCausal) mb = a.num_mblocks - 1 - mb;  // longest key ranges first
+  if (kCausal) mb = a.num_mblocks - 1 - mb;
   const int kvh = h / a.group;
 
   int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, bidx = unit;
