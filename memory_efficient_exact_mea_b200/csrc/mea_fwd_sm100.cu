@@ -9,13 +9,15 @@
 // Transformer efficienti in memoria con xFormers ...", "Applicare Attenzione
 // Causale con Maschere Inferiori", "Utilizzare Sequenze di Lunghezza Variabile").
 //
-// CTA organisation (576 threads, one CTA per SM):
+// CTA organisation (608 threads, one CTA per SM):
 //   warps 0-7   softmax / rescale / epilogue for query tile 0 (TMEM lanes 0-127):
 //               two threads per row, warps 0-3 on score columns 0-63 and the
 //               first half of the output row, warps 4-7 on the other halves
 //   warps 8-15  the same for query tile 1 (rows +128)
-//   warp  16    TMEM allocator and the single MMA-issuing thread
-//   warp  17    the single TMA-issuing thread
+//   warp  16    TMEM allocator; one thread issues every MMA of query tile 0
+//   warp  17    one thread issues every MMA of query tile 1 (the two tiles do not
+//               wait for each other: each follows its own softmax)
+//   warp  18    the single TMA-issuing thread
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
 // current key tile; P = exp(S - m) as 16-bit pairs is written back over S, each
 // 32-key chunk over its own 32 columns: fp16 P in the first 16, bf16 as P_hi in
@@ -33,9 +35,9 @@ namespace {
 
 constexpr int kBM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;        // keys per tile
-constexpr int kThreads = 576;
-constexpr int kMmaWarp = 16;
-constexpr int kTmaWarp = 17;
+constexpr int kThreads = 608;
+constexpr int kMmaWarp = 16;   // + tile: warps 16 and 17 each issue one query tile's MMAs
+constexpr int kTmaWarp = 18;
 constexpr int kSoftmaxThreadsPerTile = 256;  // two threads per row
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceeds it by < 2^8
@@ -169,14 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], kSepP ? 2 : 1);  // one release per MMA-issuing thread
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_ready[t], kSoftmaxThreadsPerTile);
       mbar_init(&o_done[t], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, kSepP ? 2 : 1);
     for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 64);
     for (int t = 0; t < 2; ++t) mbar_init(&s_free[t], kSoftmaxThreadsPerTile);
     *abort_flag = 0;
@@ -222,8 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = max(0, it - S); i < it; ++i)
         mbar_wait_drain(&kv_full[i % S], (i / S) & 1, a.status);
     }
-  } else if (warp == kMmaWarp) {
-    // ===================== MMA issuer =======================================
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ===================== MMA issuers, one per query tile ====================
+    const int tile = warp - kMmaWarp;
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_f16(BF16, kBM, kBN, false);
       const uint32_t idesc_pv = idesc_f16(BF16, kBM, D, true);
@@ -264,51 +267,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
+      // Ring index 2j holds K_j, 2j+1 holds V_j; each slot is released when both
+      // tiles' MMAs reading it have completed (two commits).  A key tile beyond
+      // this query tile's range is still waited for, so the release keeps its order.
+      // Per tile the order is Q.K_j^T, then P.V of the tile the softmax has
+      // finished: V_{j-1} in the separate-P layout (Q.K_j^T only needs S_t read out),
+      // V_j when P is written over S (Q.K_{j+1}^T must follow P.V_j).
+      const int t = tile, ntt = nt_tile[tile];
+      auto pv_step = [&](int jv) -> bool {
+        const int vs = (2 * jv + 1) % S;
+        if (!mbar_wait(&kv_full[vs], ((2 * jv + 1) / S) & 1, abort_flag, a.status)) return false;
+        MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 2);
+        if (jv < ntt) {
+          if (!mbar_wait(&p_ready[t], jv & 1, abort_flag, a.status)) return false;
+          MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 3);
+          tc_fence_after();
+          issue_pv(t, vs, jv > 0);
+          umma_commit(&o_done[t]);
+          MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 4);
+        }
+        umma_commit(&kv_empty[vs]);
+        return true;
+      };
       if (kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
-        // Ring index 2j holds K_j, 2j+1 holds V_j.  Iteration j issues Q.K_j^T
-        // for both tiles (each once its S buffer has been read out), then P.V_{j-1}.
         bool ok = true;
-        // Both tiles' MMAs go out as one batch (Q.K^T: 8 instructions, P.V: 16):
-        // every batch that starts after an idle tensor pipe pays its fill latency.
-        for (int j = 0; j <= nt && ok; ++j) {
-          if (j < nt) {
-            const int ks = (2 * j) % S;
-            if (!(ok = mbar_wait(&kv_full[ks], ((2 * j) / S) & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + j * 16 + 0);
-            if (j > 0) {  // the softmax has read S_t out of TMEM
-              for (int t = 0; t < 2 && ok; ++t)
-                if (j < nt_tile[t]) ok = mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, a.status);
-              if (!ok) break;
+        for (int j = 0; j < nt && ok; ++j) {
+          const int ks = (2 * j) % S;
+          if (!(ok = mbar_wait(&kv_full[ks], ((2 * j) / S) & 1, abort_flag, a.status))) break;
+          MEA_TRACE_AT(1024 + t * 256 + j * 8 + 0);
+          if (j < ntt) {
+            if (j > 0) {  // the softmax has read S_t(j-1) out of TMEM
+              if (!(ok = mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, a.status))) break;
               tc_fence_after();
             }
-            MEA_TRACE_AT(1024 + j * 16 + 1);
-            for (int t = 0; t < 2; ++t) {
-              if (j >= nt_tile[t]) continue;
-              issue_qk(t, ks);
-              umma_commit(&s_full[t]);
-            }
-            MEA_TRACE_AT(1024 + j * 16 + 3);
-            umma_commit(&kv_empty[ks]);
+            issue_qk(t, ks);
+            umma_commit(&s_full[t]);
+            MEA_TRACE_AT(1024 + t * 256 + j * 8 + 1);
           }
-          if (j >= 1) {
-            const int jv = j - 1, vs = (2 * jv + 1) % S;
-            if (!(ok = mbar_wait(&kv_full[vs], ((2 * jv + 1) / S) & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + j * 16 + 4);
-            for (int t = 0; t < 2 && ok; ++t)
-              if (jv < nt_tile[t]) ok = mbar_wait(&p_ready[t], jv & 1, abort_flag, a.status);
-            if (!ok) break;
-            MEA_TRACE_AT(1024 + j * 16 + 5);
-            tc_fence_after();
-            for (int t = 0; t < 2; ++t) {
-              if (jv >= nt_tile[t]) continue;
-              issue_pv(t, vs, jv > 0);
-              umma_commit(&o_done[t]);
-            }
-            MEA_TRACE_AT(1024 + j * 16 + 6);
-            umma_commit(&kv_empty[vs]);
-          }
+          umma_commit(&kv_empty[ks]);
+          if (j >= 1) ok = pv_step(j - 1);
         }
-      } else if (!kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
+        if (ok) pv_step(nt - 1);
+      }
+      // When P is written over S the chain softmax -> P.V -> Q.K^T of a tile is
+      // serial, so one thread (warp 16) issues both tiles in the interleaved
+      // order Q0.K_j, P1.V_{j-1}, Q1.K_j, P0.V_j, which keeps the two tiles half a
+      // step apart: one tile's softmax overlaps the other tile's MMAs.
+      if (!kSepP && tile == 0 && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
         int it = 0, vslot_prev = 0;
         bool ok = true;
         for (int j = 0; j < nt && ok; ++j) {
@@ -362,8 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Every MMA issued above has completed once this barrier flips.
-      umma_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, a.status);
+      if (kSepP || tile == 0) {
+        umma_commit(mma_done);
+        mbar_wait_drain(mma_done, 0, a.status);
+      }
     }
   } else {
     // ===================== softmax warpgroups ===============================
