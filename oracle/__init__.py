@@ -66,6 +66,10 @@ class Oracle:
         lib.oracle_attention_rows.restype = ctypes.c_int
         lib.oracle_attention_rows.argtypes = common + [_c_int64_p, ctypes.c_int64,
                                                        _c_double_p, _c_double_p]
+        lib.oracle_attention_bwd.restype = ctypes.c_int
+        lib.oracle_attention_bwd.argtypes = [_c_double_p] * 4 + [ctypes.c_int] * 7 + [
+            _c_int32_p, _c_int32_p, ctypes.c_int, _c_double_p, ctypes.c_double,
+            _c_double_p, _c_double_p, _c_double_p]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_int32_p,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -140,6 +144,31 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_attention_rows rejected its arguments")
         return out, lse
+
+    def attention_bwd(self, q, k, v, dout, bias=BIAS_NONE, scale=None, alibi=None,
+                      seqstart_q=None, seqstart_k=None):
+        """Gradients of sum(out * dout) -> (dq [B,M,Hq,D], dk, dv [B,N,Hkv,D])."""
+        q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+        B, M, Hq, D = q.shape
+        N, Hkv = k.shape[1], k.shape[2]
+        assert do.shape == q.shape
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        sq, sk = _i32(seqstart_q), _i32(seqstart_k)
+        if sk is None:
+            sk = sq
+        ns = 0 if sq is None else len(sq) - 1
+        slopes = self._slopes(alibi, Hq)
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        rc = self.lib.oracle_attention_bwd(
+            _ptr(q, _c_double_p), _ptr(k, _c_double_p), _ptr(v, _c_double_p),
+            _ptr(do, _c_double_p), B, M, N, Hq, Hkv, D, int(bias), _ptr(sq, _c_int32_p),
+            _ptr(sk, _c_int32_p), ns, _ptr(slopes, _c_double_p), scale,
+            _ptr(dq, _c_double_p), _ptr(dk, _c_double_p), _ptr(dv, _c_double_p))
+        if rc != 0:
+            raise ValueError("oracle_attention_bwd rejected its arguments")
+        return dq, dk, dv
 
     # -- decode --------------------------------------------------------------
     def decode(self, q, k_cache, v_cache, kv_seqstart, scale=None, alibi=None):

@@ -277,3 +277,86 @@ int oracle_decode(const double* q, const double* k_cache, const double* v_cache,
     }
     return failed ? -1 : 0;
 }
+
+/*
+ * Gradients of the attention above ("FlashAttention (2022)", section "Il trucco
+ * della softmax che non ha bisogno di vedere tutto": the backward pass recomputes
+ * the scores instead of storing them).  For one row i of query head h, with
+ * p_ij = exp(s_ij - lse_i) its softmax weights over the visible keys:
+ *     dV_j += p_ij dO_i                      dP_ij = <dO_i, v_j>
+ *     D_i   = sum_j p_ij dP_ij (= <dO_i, out_i>)
+ *     dS_ij = p_ij (dP_ij - D_i)
+ *     dQ_i  = scale sum_j dS_ij k_j          dK_j += scale dS_ij q_i
+ * dK and dV of a key/value head sum over the query heads that read it.  The
+ * bias (mask, ALiBi) does not depend on q, k or v.  Same layouts as
+ * oracle_attention; dout like out; dq like q; dk, dv like k, v.
+ */
+int oracle_attention_bwd(const double* q, const double* k, const double* v, const double* dout,
+                         int B, int M, int N, int Hq, int Hkv, int D, int bias_kind,
+                         const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+                         const double* slopes, double scale, double* dq, double* dk, double* dv) {
+    if (check_args(B, M, N, Hq, Hkv, D, bias_kind, seqstart_q, seqstart_k, num_seqs)) return -1;
+    const int group = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)B * M * Hq * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * N * Hkv * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * N * Hkv * D);
+    int failed = 0;
+    /* One (batch, kv head) per task: its dK, dV rows are written by nobody else. */
+#pragma omp parallel
+    {
+        double* p = (double*)malloc(sizeof(double) * (N > 0 ? (size_t)N : 1));
+        double* dp = (double*)malloc(sizeof(double) * (N > 0 ? (size_t)N : 1));
+        double* o = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!p || !dp || !o) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < (int64_t)B * Hkv; ++task) {
+                const int64_t b = task / Hkv;
+                const int kvh = (int)(task % Hkv);
+                for (int h = kvh * group; h < (kvh + 1) * group; ++h) {
+                    for (int64_t i = 0; i < M; ++i) {
+                        double lse;
+                        /* forward row: p holds the scores, then the weights */
+                        attention_row(q, k, v, M, N, Hq, Hkv, D, bias_kind, seqstart_q, seqstart_k,
+                                      num_seqs, slopes, scale, b, i, h, p, o, &lse);
+                        if (lse == -INFINITY) continue;  /* row sees no key: no gradient */
+                        /* attention_row left exp(s - max) (0 where masked) in p */
+                        double z = 0.0;
+                        for (int64_t j = 0; j < N; ++j) z += p[j];
+                        const double* doi = dout + ((b * M + i) * Hq + h) * D;
+                        double Di = 0.0;
+                        for (int64_t j = 0; j < N; ++j) {
+                            p[j] /= z;
+                            if (p[j] == 0.0) { dp[j] = 0.0; continue; }
+                            const double* vj = v + ((b * N + j) * Hkv + kvh) * D;
+                            double s = 0.0;
+                            for (int d = 0; d < D; ++d) s += doi[d] * vj[d];
+                            dp[j] = s;
+                            Di += p[j] * s;
+                        }
+                        const double* qi = q + ((b * M + i) * Hq + h) * D;
+                        double* dqi = dq + ((b * M + i) * Hq + h) * D;
+                        for (int64_t j = 0; j < N; ++j) {
+                            if (p[j] == 0.0) continue;
+                            const double ds = p[j] * (dp[j] - Di);
+                            const double* kj = k + ((b * N + j) * Hkv + kvh) * D;
+                            double* dkj = dk + ((b * N + j) * Hkv + kvh) * D;
+                            double* dvj = dv + ((b * N + j) * Hkv + kvh) * D;
+                            for (int d = 0; d < D; ++d) {
+                                dvj[d] += p[j] * doi[d];
+                                dqi[d] += scale * ds * kj[d];
+                                dkj[d] += scale * ds * qi[d];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+        free(o);
+    }
+    return failed ? -1 : 0;
+}

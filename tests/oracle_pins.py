@@ -354,6 +354,98 @@ def pin_brute_force(orc):
         _close(l, lb, tol=1e-10, what="brute varlen lse")
 
 
+# ---------------------------------------------------------------------------
+# Backward pass: gradients of L = sum(out * dO) with respect to q, k, v.
+# ---------------------------------------------------------------------------
+def _fd_grads(orc, q, k, v, do, eps=1e-6, **kw):
+    """Central finite differences of L through the (separately pinned) forward."""
+    def loss(q_, k_, v_):
+        return float((orc.attention(q_, k_, v_, **kw)[0] * do).sum())
+    grads = []
+    for x in (q, k, v):
+        g = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [xp if y is x else y for y in (q, k, v)]
+            args_m = [xm if y is x else y for y in (q, k, v)]
+            g[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        grads.append(g)
+    return grads
+
+
+def pin_bwd_finite_differences(orc):
+    """[flash] the recomputed-score backward equals the derivative of the forward."""
+    r = _rng(20)
+    cases = [
+        dict(shape=(1, 3, 4, 2, 1, 3), kw=dict(bias=BIAS_NONE, scale=0.7)),
+        dict(shape=(2, 4, 4, 2, 2, 3), kw=dict(bias=BIAS_CAUSAL, scale=0.5, alibi=True)),
+        dict(shape=(1, 3, 5, 4, 2, 2), kw=dict(bias=BIAS_CAUSAL, scale=1.1)),
+    ]
+    for c in cases:
+        B, M, N, Hq, Hkv, D = c["shape"]
+        q = r.standard_normal((B, M, Hq, D))
+        k, v = r.standard_normal((B, N, Hkv, D)), r.standard_normal((B, N, Hkv, D))
+        do = r.standard_normal((B, M, Hq, D))
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, **c["kw"])
+        fq, fk, fv = _fd_grads(orc, q, k, v, do, **c["kw"])
+        _close(dq, fq, tol=1e-6, what=f"fd dq {c['kw']}")
+        _close(dk, fk, tol=1e-6, what=f"fd dk {c['kw']}")
+        _close(dv, fv, tol=1e-6, what=f"fd dv {c['kw']}")
+    lens_q, lens_k = [2, 3], [3, 2]
+    q = r.standard_normal((1, 5, 2, 2))
+    k, v = r.standard_normal((1, 5, 2, 2)), r.standard_normal((1, 5, 2, 2))
+    do = r.standard_normal((1, 5, 2, 2))
+    for bias in (BIAS_BLOCKDIAG, BIAS_BLOCKDIAG_CAUSAL):
+        kw = dict(bias=bias, seqstart_q=_offsets(lens_q), seqstart_k=_offsets(lens_k), scale=0.8)
+        got = orc.attention_bwd(q, k, v, do, **kw)
+        for g, f, n in zip(got, _fd_grads(orc, q, k, v, do, **kw), "qkv"):
+            _close(g, f, tol=1e-6, what=f"fd d{n} varlen bias={bias}")
+
+
+def pin_bwd_closed_forms(orc):
+    """One key: weights are 1, so dq = dk = 0 and dv = sum of dO over the rows and
+    query heads reading it.  Constant values: dP_ij = D_i, so dS = 0 (dq = dk = 0)
+    and sum_j dv_j = sum_i dO_i."""
+    r = _rng(21)
+    q = r.standard_normal((2, 4, 4, 3))
+    k, v = r.standard_normal((2, 1, 2, 3)), r.standard_normal((2, 1, 2, 3))
+    do = r.standard_normal((2, 4, 4, 3))
+    dq, dk, dv = orc.attention_bwd(q, k, v, do, scale=0.9)
+    _close(dq, np.zeros_like(dq), what="one key dq")
+    _close(dk, np.zeros_like(dk), what="one key dk")
+    _close(dv[:, 0], do.reshape(2, 4, 2, 2, 3).sum(axis=(1, 3)), what="one key dv")
+    k = r.standard_normal((1, 6, 1, 3))
+    v = np.broadcast_to(r.standard_normal(3), (1, 6, 1, 3)).copy()
+    q, do = r.standard_normal((1, 5, 2, 3)), r.standard_normal((1, 5, 2, 3))
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, bias=bias, alibi=True)
+        _close(dq, np.zeros_like(dq), tol=1e-10, what="const v dq")
+        _close(dk, np.zeros_like(dk), tol=1e-10, what="const v dk")
+        _close(dv.sum(axis=1)[0, 0], do.sum(axis=(0, 1, 2)), tol=1e-10, what="const v sum dv")
+
+
+def pin_bwd_gqa_and_key_shift(orc):
+    """GQA gradients = those of repeated kv heads, with dk/dv summed over each
+    group; adding one vector to every key leaves dq and dv unchanged (each row
+    of dS sums to zero)."""
+    r = _rng(22)
+    q, do = r.standard_normal((1, 4, 4, 3)), r.standard_normal((1, 4, 4, 3))
+    k, v = r.standard_normal((1, 5, 2, 3)), r.standard_normal((1, 5, 2, 3))
+    a = orc.attention_bwd(q, k, v, do, bias=BIAS_CAUSAL, alibi=True)
+    b = orc.attention_bwd(q, np.repeat(k, 2, axis=2), np.repeat(v, 2, axis=2), do,
+                          bias=BIAS_CAUSAL, alibi=True)
+    _close(a[0], b[0], tol=1e-10, what="gqa dq")
+    _close(a[1], b[1].reshape(1, 5, 2, 2, 3).sum(axis=3), tol=1e-10, what="gqa dk")
+    _close(a[2], b[2].reshape(1, 5, 2, 2, 3).sum(axis=3), tol=1e-10, what="gqa dv")
+    c = orc.attention_bwd(q, k + r.standard_normal(3), v, do, bias=BIAS_CAUSAL, alibi=True)
+    _close(c[0], a[0], tol=1e-9, what="key shift dq")
+    _close(c[2], a[2], tol=1e-9, what="key shift dv")
+
+
 PINS = [
     pin_weights_sum_to_one,
     pin_causal_row0_is_v0,
@@ -369,4 +461,7 @@ PINS = [
     pin_key_shift_invariance,
     pin_rows_match_full,
     pin_brute_force,
+    pin_bwd_finite_differences,
+    pin_bwd_closed_forms,
+    pin_bwd_gqa_and_key_shift,
 ]

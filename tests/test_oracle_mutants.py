@@ -30,6 +30,12 @@ MUTANTS = [
     ("decode_gqa_modulo", "kvh = h / group;", "kvh = h % Hkv;", 1),
     ("decode_lse_without_max", "lse[r] = mx + log(z);", "lse[r] = log(z);", 0),
     ("decode_value_from_key", "const double* vj = v_cache +", "const double* vj = k_cache +", 0),
+    ("bwd_without_row_term", "const double ds = p[j] * (dp[j] - Di);",
+     "const double ds = p[j] * dp[j];", 0),
+    ("bwd_dk_from_key", "dkj[d] += scale * ds * qi[d];", "dkj[d] += scale * ds * kj[d];", 0),
+    ("bwd_dq_unscaled", "dqi[d] += scale * ds * kj[d];", "dqi[d] += ds * kj[d];", 0),
+    ("bwd_dv_from_dp", "dvj[d] += p[j] * doi[d];", "dvj[d] += dp[j] * doi[d];", 0),
+    ("bwd_unnormalised", "p[j] /= z;", "p[j] /= 1.0;", 0),
 ]
 
 
