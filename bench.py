@@ -276,6 +276,10 @@ def run_ours(args, rank, world, local):
         also["causal_small"] = measure_prefill(mea, synth.causal_small(), dev, stream, tc_peak,
                                                iters=50)
         also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
+        also["bwd_noncausal_m2048"] = measure_backward(mea, synth.noncausal_sweep(2048), dev,
+                                                       stream, tc_peak)
+        also["bwd_gqa_alibi_causal"] = measure_backward(mea, synth.gqa_alibi_causal(), dev,
+                                                        stream, tc_peak)
     assert mea.read_device_status() == 0
 
     traffic = traffic_for("fwd_sweep")
@@ -431,6 +435,32 @@ def measure_prefill(mea, p, dev, stream, tc_peak, iters=10):
             "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor"}
 
 
+def measure_backward(mea, p, dev, stream, tc_peak, iters=5):
+    """mea_bwd alone (the forward that makes out and lse runs once, untimed).
+    Work: five contractions of 2*K FLOP per visible (query, key) pair -- S, dP,
+    dV, dK, dQ -- i.e. 2.5x the forward's count."""
+    q, k, v = p.q.to(dev), p.k.to(dev), p.v.to(dev)
+    kw = {}
+    if p.seq_lens_q is not None:
+        kw = dict(seqstart_q=p.seqstart_q.to(dev), seqstart_k=p.seqstart_k.to(dev),
+                  max_seqlen_q=max(p.seq_lens_q),
+                  max_seqlen_k=max(p.seq_lens_k or p.seq_lens_q))
+    g = synth.generator(p.seed + 17)
+    dout = synth.randn(tuple(p.q.shape), p.dtype, g).to(dev)
+    out, lse = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, **kw)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    B, M, Hq, K = q.shape
+    ws = torch.empty(mea.lib.mea_bwd_workspace_size(B, M, Hq, K), dtype=torch.uint8, device=dev)
+    ms = _time(lambda: mea.mea_bwd(q, k, v, out, dout, lse, bias=p.bias, scale=p.scale,
+                                   alibi=p.alibi, dq=dq, dk=dk, dv=dv, workspace=ws, **kw),
+               stream, iters)
+    f = 2.5 * prefill_flops(p)
+    tf = f / (ms * 1e-3) / 1e12
+    return {"workload": "bwd_" + p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
+            "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor",
+            "kernel": "mma.sync m16n8k16 (legacy tensor path)"}
+
+
 def measure_decode(mea, d, dev, stream, hbm_peak, iters=20):
     q, kc, vc = d.q.to(dev), d.k_cache.to(dev), d.v_cache.to(dev)
     st = d.kv_seqstart.to(dev)
@@ -506,6 +536,7 @@ PROFILE_CASES = {
     "fwd_sweep_m2048": lambda: ("fwd", synth.noncausal_sweep(2048)),
     "fwd_gqa_alibi_m2048": lambda: ("fwd", synth.gqa_alibi_causal(M=2048, B=2)),
     "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
+    "bwd_m2048": lambda: ("bwd", synth.noncausal_sweep(2048)),
     "decode_b16": lambda: ("decode", synth.make_decode(
         "decode_b16", synth.decode_lengths()[:16], 32, 8, 128, "bf16", seed=1005)),
 }
@@ -532,6 +563,13 @@ def run_profile(args):
 
         def fn():
             mea.mea_fwd(q, k, v, bias=w.bias, scale=w.scale, alibi=w.alibi, **kw)
+    elif kind == "bwd":
+        q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
+        dout = synth.randn(tuple(w.q.shape), w.dtype, synth.generator(w.seed + 17)).to(dev)
+        out, lse = mea.mea_fwd(q, k, v, bias=w.bias, scale=w.scale, alibi=w.alibi)
+
+        def fn():
+            mea.mea_bwd(q, k, v, out, dout, lse, bias=w.bias, scale=w.scale, alibi=w.alibi)
     else:
         q, kc, vc = w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev)
         st = w.kv_seqstart.to(dev)

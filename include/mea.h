@@ -179,6 +179,46 @@ int mea_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                        int B, int Hq, int Hkv, int K, int cache_rows, int max_kv_len,
                        mea_dtype_t dtype, int alibi, float scale, cudaStream_t stream);
 
+/*
+ * mea_bwd -- gradients of the attention of mea_fwd ("FlashAttention (2022)",
+ * section "Il trucco della softmax che non ha bisogno di vedere tutto": the
+ * backward pass recomputes the attention weights from q, k and the forward's
+ * log-sum-exp instead of reading a stored score matrix).  With
+ * p_ij = exp(scale q_i.k_j + b_ij - lse_i) and D_i = <dout_i, out_i>:
+ *     dv_j = sum_i p_ij dout_i            dP_ij = <dout_i, v_j>
+ *     dS_ij = p_ij (dP_ij - D_i)
+ *     dq_i = scale sum_j dS_ij k_j        dk_j = scale sum_i dS_ij q_i
+ * dk and dv of a key/value head sum over the Hq/Hkv query heads that read it.
+ *
+ *   q, out, dout, dq  [B, M, Hq, K]  contiguous, dtype `dtype`
+ *   k, v, dk, dv      [B, N, Hkv, K] contiguous, dtype `dtype`
+ *   lse               [B, Hq, M] fp32 natural log, as written by mea_fwd for the
+ *                     same q, k, v, bias and scale (-inf for rows that see no key)
+ *   bias, seqstart_q, seqstart_k, num_seqs, max_seqlen_k, alibi, scale: as for
+ *   mea_fwd (max_seqlen_q is accepted for symmetry and unused).
+ *
+ * dq, dk, dv are written in full (rows that see no key, and keys no query sees,
+ * get 0).  The outputs must not alias the inputs.
+ *
+ * workspace: DEVICE scratch of at least mea_bwd_workspace_size(B, M, Hq, K)
+ * bytes, 256-byte aligned, owned by the caller, holding an fp32 dq accumulator
+ * and D; it needs no initialisation and is garbage afterwards.  Calls that share
+ * a workspace must not overlap.  Too small or misaligned: MEA_ERR_WORKSPACE.
+ * Non-contiguous layouts are not accepted by this entry point (pass contiguous
+ * copies); pointers not 16-byte aligned give MEA_ERR_UNSUPPORTED.
+ * Returns MEA_OK or an error status; never synchronises.
+ */
+size_t mea_bwd_workspace_size(int B, int M, int Hq, int K);
+
+int mea_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+            const float* lse, void* dq, void* dk, void* dv,
+            int B, int M, int N, int Hq, int Hkv, int K,
+            mea_dtype_t dtype, mea_bias_t bias,
+            const int32_t* seqstart_q, const int32_t* seqstart_k,
+            int num_seqs, int max_seqlen_q, int max_seqlen_k,
+            int alibi, float scale, void* workspace, size_t workspace_bytes,
+            cudaStream_t stream);
+
 /* Number of key/value rows one decode split covers (the unit of parallelism). */
 int mea_decode_chunk(void);
 

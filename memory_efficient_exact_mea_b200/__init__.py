@@ -17,7 +17,7 @@ import os
 
 import torch
 
-__all__ = ["mea_fwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
+__all__ = ["mea_fwd", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
            "read_device_status", "status_string", "MeaError", "BIAS", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
@@ -48,6 +48,10 @@ def _load() -> ctypes.CDLL:
     L.mea_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.mea_decode.restype = i
     L.mea_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.mea_bwd_workspace_size.restype = sz
+    L.mea_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.mea_bwd.restype = i
+    L.mea_bwd.argtypes = [vp] * 9 + [i] * 8 + [vp, vp, i, i, i, i, f, vp, sz, vp]
     L.mea_decode_chunk.restype = i
     L.mea_decode_chunk.argtypes = []
     L.mea_status_string.restype = ctypes.c_char_p
@@ -137,6 +141,47 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
                      scale, _stream(stream))
     _check("mea_fwd", rc)
     return out, lse
+
+
+def mea_bwd(q, k, v, out, dout, lse, bias: str = "none", scale: float | None = None,
+            alibi: bool = False, seqstart_q=None, seqstart_k=None,
+            max_seqlen_q: int | None = None, max_seqlen_k: int | None = None,
+            dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Attention backward.  Contiguous q/out/dout [B,M,Hq,K], k/v [B,N,Hkv,K] and the
+    forward's lse [B,Hq,M] -> (dq, dk, dv) shaped like q, k, v."""
+    B, M, Hq, K = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.dtype not in _DTYPE or any(t.dtype != q.dtype for t in (k, v, out, dout)):
+        raise ValueError("q, k, v, out, dout must share dtype float16 or bfloat16")
+    scale = K ** -0.5 if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = int(lib.mea_bwd_workspace_size(B, M, Hq, K))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    kind = BIAS[bias]
+    ns = 0
+    if kind >= 2:
+        ns = seqstart_q.numel() - 1
+        if max_seqlen_q is None:
+            max_seqlen_q = int(torch.diff(seqstart_q).max().item()) if ns > 0 else 0
+        if max_seqlen_k is None:
+            sk = seqstart_q if seqstart_k is None else seqstart_k
+            max_seqlen_k = int(torch.diff(sk).max().item()) if ns > 0 else 0
+    else:
+        seqstart_q = seqstart_k = None
+        max_seqlen_q = max_seqlen_k = 0
+    rc = lib.mea_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq),
+                     _ptr(dk), _ptr(dv), B, M, N, Hq, Hkv, K, _DTYPE[q.dtype], kind,
+                     _ptr(seqstart_q), _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k),
+                     int(bool(alibi)), scale, _ptr(workspace), ws_bytes, _stream(stream))
+    _check("mea_bwd", rc)
+    return dq, dk, dv
 
 
 def mea_decode_workspace_size(B: int, Hq: int, Hkv: int, K: int, max_kv_len: int) -> int:

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["mea_api.cu", "mea_fwd_sm100.cu", "mea_decode_sm100.cu"]
+SOURCES = ["mea_api.cu", "mea_fwd_sm100.cu", "mea_decode_sm100.cu", "mea_bwd_sm100.cu"]
 LIB = os.path.join(HERE, "libmea.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -281,3 +281,89 @@ extern "C" int mea_selftest_timeout(int timeout_us, cudaStream_t stream) {
   selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, 1000ull * timeout_us);
   return cudaGetLastError() == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Backward
+// ---------------------------------------------------------------------------
+extern "C" size_t mea_bwd_workspace_size(int B, int M, int Hq, int K) {
+  if (B < 0 || M < 0 || Hq <= 0 || K <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * M * Hq;
+  return align256(rows * K * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int M, int N, int Hq, int Hkv, int K, mea_dtype_t dtype, mea_bias_t bias,
+                       const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+                       int max_seqlen_q, int max_seqlen_k, int alibi, float scale,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  (void)max_seqlen_q;
+  if (B < 0 || M < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return MEA_ERR_INVALID_ARG;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
+  if (bias < MEA_BIAS_NONE || bias > MEA_BIAS_BLOCKDIAG_CAUSAL) return MEA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return MEA_ERR_INVALID_ARG;
+  if (B == 0 || (M == 0 && N == 0)) return MEA_OK;
+  if ((M > 0 && (!q || !out || !dout || !lse || !dq)) || (N > 0 && (!k || !v || !dk || !dv)))
+    return MEA_ERR_INVALID_ARG;
+  if (K != 64 && K != 128) return MEA_ERR_UNSUPPORTED;
+  const bool packed = bias == MEA_BIAS_BLOCKDIAG || bias == MEA_BIAS_BLOCKDIAG_CAUSAL;
+  if (packed) {
+    if (B != 1 || !seqstart_q || num_seqs <= 0 || max_seqlen_k < 0) return MEA_ERR_INVALID_ARG;
+    if (!seqstart_k && M != N) return MEA_ERR_INVALID_ARG;
+  }
+  for (const void* p : {q, k, v, out, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if (p && !aligned16(p)) return MEA_ERR_UNSUPPORTED;
+  const size_t need = mea_bwd_workspace_size(B, M, Hq, K);
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return MEA_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return MEA_ERR_CUDA;
+
+  mea::BwdLaunch L{};
+  mea::BwdArgs& a = L.args;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  const size_t rows = static_cast<size_t>(B) * M * Hq;
+  a.dq_acc = static_cast<float*>(workspace);
+  a.delta = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                     align256(rows * K * sizeof(float)));
+  a.seqstart_q = packed ? seqstart_q : nullptr;
+  a.seqstart_k = packed ? (seqstart_k ? seqstart_k : seqstart_q) : nullptr;
+  a.status = status;
+  a.B = B;
+  a.M = M;
+  a.N = N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.num_units = packed ? num_seqs : B;
+  const int krows = packed ? max_seqlen_k : N;
+  a.num_kblocks = (krows + mea::kBwdBlock - 1) / mea::kBwdBlock;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  L.head_dim = K;
+  L.bf16 = dtype == MEA_BF16;
+  L.mask = static_cast<int>(bias);
+  L.alibi = alibi != 0;
+  if (N > 0 && M == 0) {  // no query rows: dk = dv = 0
+    if (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess)
+      return MEA_ERR_CUDA;
+    return MEA_OK;
+  }
+  if (N > 0 && (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) !=
+                    cudaSuccess ||
+                cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) !=
+                    cudaSuccess))
+    return MEA_ERR_CUDA;
+  return mea::launch_bwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}

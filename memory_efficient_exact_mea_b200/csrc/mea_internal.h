@@ -64,4 +64,30 @@ struct DecodeLaunch {
 
 cudaError_t launch_decode(const DecodeLaunch& launch, cudaStream_t stream);
 
+// Backward: dq, dk, dv from q, k, v, out, dout and the forward's lse.
+constexpr int kBwdBlock = 64;  // query rows and key rows per tile
+
+struct BwdArgs {
+  const void *q, *k, *v, *out, *dout;  // contiguous [B,M,Hq,K] / [B,N,Hkv,K]
+  const float* lse;                    // [B, Hq, M] natural log (from mea_fwd)
+  void *dq, *dk, *dv;
+  float* dq_acc;                       // [B, M, Hq, K] fp32 workspace
+  float* delta;                        // [B, Hq, M] fp32 workspace: <dout_i, out_i>
+  const int32_t* seqstart_q;
+  const int32_t* seqstart_k;
+  int* status;
+  int B, M, N, Hq, Hkv, group, num_units, num_kblocks;
+  float scale, scale_log2;
+};
+
+struct BwdLaunch {
+  BwdArgs args;
+  int head_dim;
+  bool bf16;
+  int mask;
+  bool alibi;
+};
+
+cudaError_t launch_bwd(const BwdLaunch& launch, cudaStream_t stream);
+
 }  // namespace mea

@@ -136,3 +136,46 @@ def test_no_device_is_reported_not_crashed(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _fwd(lib) == -4
+
+
+def _bwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, out=16, do=16, lse=16, dq=16, dk=16, dv=16, B=2, M=100, N=100,
+             Hq=8, Hkv=2, K=128, dtype=1, bias=1, sq=None, sk=None, ns=0, msq=0, msk=0, alibi=0,
+             scale=0.1, ws=256, wsb=1 << 30, stream=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return lib.mea_bwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["out"]), vp(a["do"]),
+                       vp(a["lse"]), vp(a["dq"]), vp(a["dk"]), vp(a["dv"]), a["B"], a["M"],
+                       a["N"], a["Hq"], a["Hkv"], a["K"], a["dtype"], a["bias"], vp(a["sq"]),
+                       vp(a["sk"]), a["ns"], a["msq"], a["msk"], a["alibi"],
+                       ctypes.c_float(a["scale"]), vp(a["ws"]), a["wsb"], vp(a["stream"]))
+
+
+def test_bwd_workspace_size():
+    import memory_efficient_exact_mea_b200 as m
+
+    r256 = lambda x: -(-x // 256) * 256  # noqa: E731
+    for (B, M, Hq, K) in ((2, 100, 8, 128), (1, 1, 1, 64), (4, 4096, 32, 128)):
+        rows = B * M * Hq
+        assert m.lib.mea_bwd_workspace_size(B, M, Hq, K) == r256(rows * K * 4) + r256(rows * 4)
+    assert m.lib.mea_bwd_workspace_size(-1, 4, 4, 64) == 0
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    INVALID, UNSUPPORTED, WORKSPACE = -1, -2, -3
+    assert _bwd(lib, Hq=3, Hkv=2) == INVALID
+    assert _bwd(lib, N=-1) == INVALID
+    assert _bwd(lib, dtype=5) == INVALID
+    assert _bwd(lib, bias=4) == INVALID
+    assert _bwd(lib, scale=float("nan")) == INVALID
+    assert _bwd(lib, lse=None) == INVALID
+    assert _bwd(lib, dk=None) == INVALID
+    assert _bwd(lib, bias=2) == INVALID                   # block-diagonal needs B == 1 ...
+    assert _bwd(lib, bias=3, B=1, ns=1) == INVALID         # ... and offsets
+    assert _bwd(lib, K=32) == UNSUPPORTED
+    assert _bwd(lib, dq=40) == UNSUPPORTED                 # 16-byte alignment
+    assert _bwd(lib, ws=None) == WORKSPACE
+    assert _bwd(lib, wsb=1024) == WORKSPACE
+    assert _bwd(lib, ws=512 + 16) == WORKSPACE             # 256-byte alignment
+    assert _bwd(lib, B=0) == 0
+    assert _bwd(lib, M=0, N=0) == 0
