@@ -22,7 +22,9 @@
 // current key tile; P = exp(S - m) as 16-bit pairs is written back over S, each
 // 32-key chunk over its own 32 columns: fp16 P in the first 16, bf16 as P_hi in
 // the first 16 and P_lo = P - P_hi in the last 16; the P.V MMA reads P straight
-// from TMEM) | O0 | O1 (K columns each, the fp32 output accumulators).
+// from TMEM) | O0 | O1 (K columns each, the fp32 output accumulators).  At K = 64
+// with fp16, P has columns of its own instead (S0 | S1 | P0 | P1 | O0 | O1 =
+// 128 + 128 + 64 + 64 + 64 + 64), so each tile's next Q.K^T overlaps its softmax.
 // Shared memory: Q0, Q1 (loaded once) and a ring of key/value tiles, all in the
 // 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
