@@ -23,6 +23,7 @@ BIAS_NONE, BIAS_CAUSAL, BIAS_BLOCKDIAG, BIAS_BLOCKDIAG_CAUSAL = 0, 1, 2, 3
 _c_double_p = ctypes.POINTER(ctypes.c_double)
 _c_int32_p = ctypes.POINTER(ctypes.c_int32)
 _c_int64_p = ctypes.POINTER(ctypes.c_int64)
+_c_uint8_p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def _f64(x) -> np.ndarray:
@@ -70,6 +71,10 @@ class Oracle:
         lib.oracle_attention_bwd.argtypes = [_c_double_p] * 4 + [ctypes.c_int] * 7 + [
             _c_int32_p, _c_int32_p, ctypes.c_int, _c_double_p, ctypes.c_double,
             _c_double_p, _c_double_p, _c_double_p]
+        lib.oracle_attention_block_sparse.restype = ctypes.c_int
+        lib.oracle_attention_block_sparse.argtypes = [_c_double_p] * 3 + [ctypes.c_int] * 7 + [
+            _c_uint8_p, ctypes.c_int, ctypes.c_int, _c_double_p, ctypes.c_double, _c_int64_p,
+            ctypes.c_int64, _c_double_p, _c_double_p]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_int32_p,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -169,6 +174,42 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_attention_bwd rejected its arguments")
         return dq, dk, dv
+
+    def attention_block_sparse(self, q, k, v, block_mask, block_m, block_n, bias=BIAS_NONE,
+                               scale=None, alibi=None, rows=None):
+        """Block-sparse attention.  block_mask: uint8 [B, Hq, ceil(M/block_m),
+        ceil(N/block_n)] (0 = block left out).  rows None -> (out [B,M,Hq,D],
+        lse [B,Hq,M]); rows int [n, 3] of (b, i, h) -> (out [n, D], lse [n])."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, M, Hq, D = q.shape
+        N, Hkv = k.shape[1], k.shape[2]
+        assert k.shape == (B, N, Hkv, D) and v.shape == k.shape
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        mask = block_mask
+        if hasattr(mask, "detach"):
+            mask = mask.detach().to("cpu").numpy()
+        mask = np.ascontiguousarray(np.asarray(mask, dtype=np.uint8))
+        mb, nb = -(-M // block_m), -(-N // block_n)
+        assert mask.shape == (B, Hq, mb, nb), (mask.shape, (B, Hq, mb, nb))
+        slopes = self._slopes(alibi, Hq)
+        if rows is None:
+            out = np.zeros((B, M, Hq, D), dtype=np.float64)
+            lse = np.zeros((B, Hq, M), dtype=np.float64)
+            rows_p, n = None, 0
+        else:
+            rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+            n = rows.shape[0]
+            out = np.zeros((n, D), dtype=np.float64)
+            lse = np.zeros((n,), dtype=np.float64)
+            rows_p = _ptr(rows, _c_int64_p)
+        rc = self.lib.oracle_attention_block_sparse(
+            _ptr(q, _c_double_p), _ptr(k, _c_double_p), _ptr(v, _c_double_p),
+            B, M, N, Hq, Hkv, D, int(bias), _ptr(mask, _c_uint8_p), int(block_m), int(block_n),
+            _ptr(slopes, _c_double_p), scale, rows_p, n,
+            _ptr(out, _c_double_p), _ptr(lse, _c_double_p))
+        if rc != 0:
+            raise ValueError("oracle_attention_block_sparse rejected its arguments")
+        return out, lse
 
     # -- decode --------------------------------------------------------------
     def decode(self, q, k_cache, v_cache, kv_seqstart, scale=None, alibi=None):

@@ -73,13 +73,15 @@ static int find_seq(const int32_t* start, int num_seqs, int64_t r) {
 /*
  * One output row: query row i of batch b, query head h.  Writes D values to
  * out_row and one value to *lse_row.  `score` is caller scratch of N doubles.
+ * `keep` (NULL: no block mask) is this row's row of a block mask: key j is
+ * visible only if keep[j / block_n] is nonzero.
  */
 static void attention_row(const double* q, const double* k, const double* v,
                           int M, int N, int Hq, int Hkv, int D, int bias_kind,
                           const int32_t* seqstart_q, const int32_t* seqstart_k,
                           int num_seqs, const double* slopes, double scale,
-                          int64_t b, int64_t i, int h, double* score,
-                          double* out_row, double* lse_row) {
+                          int64_t b, int64_t i, int h, const uint8_t* keep, int64_t block_n,
+                          double* score, double* out_row, double* lse_row) {
     const int group = Hq / Hkv;
     const int kvh = h / group;
     const double* qi = q + ((b * M + i) * Hq + h) * D;
@@ -107,6 +109,7 @@ static void attention_row(const double* q, const double* k, const double* v,
         int64_t pos_j = j - j_lo;
         int visible = (j >= j_lo && j < j_hi);
         if (causal && pos_j > pos_i) visible = 0;
+        if (keep && !keep[j / block_n]) visible = 0;
         if (!visible) { score[j] = -INFINITY; continue; }
         const double* kj = k + ((b * N + j) * Hkv + kvh) * D;
         double dot = 0.0;
@@ -176,7 +179,7 @@ int oracle_attention_rows(const double* q, const double* k, const double* v,
             for (int64_t r = 0; r < n_rows; ++r) {
                 attention_row(q, k, v, M, N, Hq, Hkv, D, bias_kind, seqstart_q, seqstart_k,
                               num_seqs, slopes, scale, rows[3 * r], rows[3 * r + 1],
-                              (int)rows[3 * r + 2], score, out + r * D, lse + r);
+                              (int)rows[3 * r + 2], NULL, 1, score, out + r * D, lse + r);
             }
             free(score);
         }
@@ -206,9 +209,69 @@ int oracle_attention(const double* q, const double* k, const double* v,
                 const int h = (int)(r % Hq);
                 double lse_val;
                 attention_row(q, k, v, M, N, Hq, Hkv, D, bias_kind, seqstart_q, seqstart_k,
-                              num_seqs, slopes, scale, b, i, h, score,
+                              num_seqs, slopes, scale, b, i, h, NULL, 1, score,
                               out + ((b * M + i) * Hq + h) * D, &lse_val);
                 lse[(b * Hq + h) * M + i] = lse_val;
+            }
+            free(score);
+        }
+    }
+    return failed ? -1 : 0;
+}
+
+/*
+ * Block-sparse attention ("FlashAttention (2022)", section "Cosa mostravano i
+ * numeri", which names the block-sparse variant of the method): the score
+ * matrix of each (batch, query head) is cut into block_m x block_n blocks and
+ * a block whose mask entry is zero is left out, i.e. its scores are -inf, on
+ * top of the bias kind (none or causal).  The result is the dense definition
+ * above with that mask; a row left with no visible key has out = 0, lse = -inf.
+ *   block_mask  uint8 [B, Hq, ceil(M / block_m), ceil(N / block_n)], contiguous;
+ *               query row i, key j of (b, h) use entry
+ *               [b][h][i / block_m][j / block_n].
+ * rows (n_rows triples (b, i, h)) selects rows as in oracle_attention_rows,
+ * with out [n_rows, D] and lse [n_rows]; rows == NULL computes every row into
+ * out [B, M, Hq, D] and lse [B, Hq, M].
+ */
+int oracle_attention_block_sparse(const double* q, const double* k, const double* v,
+                                  int B, int M, int N, int Hq, int Hkv, int D, int bias_kind,
+                                  const uint8_t* block_mask, int block_m, int block_n,
+                                  const double* slopes, double scale,
+                                  const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    if (check_args(B, M, N, Hq, Hkv, D, bias_kind, NULL, NULL, 0)) return -1;
+    if (bias_kind != ORACLE_BIAS_NONE && bias_kind != ORACLE_BIAS_CAUSAL) return -1;
+    if (!block_mask || block_m <= 0 || block_n <= 0) return -1;
+    const int64_t mblocks = (M + block_m - 1) / block_m, nblocks = (N + block_n - 1) / block_n;
+    const int64_t total = rows ? n_rows : (int64_t)B * M * Hq;
+    for (int64_t r = 0; rows && r < n_rows; ++r) {
+        const int64_t b = rows[3 * r], i = rows[3 * r + 1], h = rows[3 * r + 2];
+        if (b < 0 || b >= B || i < 0 || i >= M || h < 0 || h >= Hq) return -1;
+    }
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* score = (double*)malloc(sizeof(double) * (N > 0 ? (size_t)N : 1));
+        if (!score) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t r = 0; r < total; ++r) {
+                int64_t b, i;
+                int h;
+                if (rows) {
+                    b = rows[3 * r]; i = rows[3 * r + 1]; h = (int)rows[3 * r + 2];
+                } else {
+                    b = r / ((int64_t)M * Hq); i = (r / Hq) % M; h = (int)(r % Hq);
+                }
+                const uint8_t* keep =
+                    block_mask + (((b * Hq + h) * mblocks) + i / block_m) * nblocks;
+                double* orow = rows ? out + r * D : out + ((b * M + i) * Hq + h) * D;
+                double lse_val;
+                attention_row(q, k, v, M, N, Hq, Hkv, D, bias_kind, NULL, NULL, 0, slopes,
+                              scale, b, i, h, keep, block_n, score, orow, &lse_val);
+                if (rows) lse[r] = lse_val;
+                else lse[(b * Hq + h) * M + i] = lse_val;
             }
             free(score);
         }
@@ -320,7 +383,7 @@ int oracle_attention_bwd(const double* q, const double* k, const double* v, cons
                         double lse;
                         /* forward row: p holds the scores, then the weights */
                         attention_row(q, k, v, M, N, Hq, Hkv, D, bias_kind, seqstart_q, seqstart_k,
-                                      num_seqs, slopes, scale, b, i, h, p, o, &lse);
+                                      num_seqs, slopes, scale, b, i, h, NULL, 1, p, o, &lse);
                         if (lse == -INFINITY) continue;  /* row sees no key: no gradient */
                         /* attention_row left exp(s - max) (0 where masked) in p */
                         double z = 0.0;

@@ -15,6 +15,8 @@ Passages (page title, section):
             causal lower-triangular mask, block-diagonal packed sequences, GQA, ALiBi
   [flash]   "FlashAttention (2022)", "Il trucco della softmax ...": softmax weights
             of a row sum to one; the result is exact.
+  [sparse]  "FlashAttention (2022)", "Cosa mostravano i numeri": the block-sparse
+            variant leaves out whole blocks of the score matrix; exact otherwise.
 """
 from __future__ import annotations
 
@@ -446,6 +448,104 @@ def pin_bwd_gqa_and_key_shift(orc):
     _close(c[2], a[2], tol=1e-9, what="key shift dv")
 
 
+# ---------------------------------------------------------------------------
+# [sparse] block-sparse attention = the dense definition with a block mask.
+# ---------------------------------------------------------------------------
+def pin_block_sparse_reductions(orc):
+    """All-ones mask = the dense run; a diagonal block mask = the block-diagonal
+    run of the same chunks (rectangular blocks fix which axis is which); under
+    causal with square blocks and M = N, = the block-diagonal causal run; a row
+    whose blocks are all zero gets out = 0, lse = -inf."""
+    r = _rng(30)
+    B, M, N, Hq, Hkv, D = 2, 7, 9, 4, 2, 5
+    q = r.standard_normal((B, M, Hq, D))
+    k, v = r.standard_normal((B, N, Hkv, D)), r.standard_normal((B, N, Hkv, D))
+    bm, bn = 2, 4
+    ones = np.ones((B, Hq, -(-M // bm), -(-N // bn)), dtype=np.uint8)
+    for bias in (BIAS_NONE, BIAS_CAUSAL):
+        o, l = orc.attention_block_sparse(q, k, v, ones, bm, bn, bias=bias, alibi=True)
+        od, ld = orc.attention(q, k, v, bias=bias, alibi=True)
+        _close(o, od, what="all-ones mask out")
+        _close(l, ld, what="all-ones mask lse")
+    # diagonal: query chunks of 2 rows against key chunks of 3 keys
+    q1 = r.standard_normal((1, 6, 2, 4))
+    k1, v1 = r.standard_normal((1, 9, 2, 4)), r.standard_normal((1, 9, 2, 4))
+    diag = np.broadcast_to(np.eye(3, dtype=np.uint8), (1, 2, 3, 3)).copy()
+    o, l = orc.attention_block_sparse(q1, k1, v1, diag, 2, 3, scale=0.7)
+    ob, lb = orc.attention(q1, k1, v1, bias=BIAS_BLOCKDIAG, seqstart_q=_offsets([2, 2, 2]),
+                           seqstart_k=_offsets([3, 3, 3]), scale=0.7)
+    _close(o, ob, what="diagonal mask = blockdiag out")
+    _close(l, lb, what="diagonal mask = blockdiag lse")
+    q2 = r.standard_normal((1, 9, 2, 4))
+    o, l = orc.attention_block_sparse(q2, k1, v1, diag, 3, 3, bias=BIAS_CAUSAL, scale=0.7)
+    ob, lb = orc.attention(q2, k1, v1, bias=BIAS_BLOCKDIAG_CAUSAL, seqstart_q=_offsets([3, 3, 3]),
+                           seqstart_k=_offsets([3, 3, 3]), scale=0.7)
+    _close(o, ob, what="diagonal causal mask out")
+    _close(l, lb, what="diagonal causal mask lse")
+    holes = ones.copy()
+    holes[1, 3, 2, :] = 0  # rows 4, 5 of (b=1, h=3) see nothing
+    o, l = orc.attention_block_sparse(q, k, v, holes, bm, bn)
+    _close(o[1, 4:6, 3], np.zeros((2, D)), what="empty block row out")
+    assert np.all(np.isneginf(l[1, 3, 4:6])), "empty block row lse"
+    od, ld = orc.attention(q, k, v)
+    _close(o[0], od[0], what="other rows untouched")
+
+
+def brute_force_block_sparse(q, k, v, mask, bm, bn, causal, scale):
+    """Full score matrix with the block mask expanded element by element."""
+    B, M, Hq, D = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    out = np.zeros((B, M, Hq, D))
+    lse = np.full((B, Hq, M), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            allowed = np.kron(mask[b, h], np.ones((bm, bn)))[:M, :N] > 0
+            if causal:
+                allowed &= np.arange(N)[None, :] <= np.arange(M)[:, None] + (N - M)
+            S = np.where(allowed, scale * (q[b, :, h] @ k[b, :, h // G].T), -np.inf)
+            for i in range(M):
+                if allowed[i].any():
+                    m = S[i].max()
+                    e = np.exp(S[i] - m)
+                    out[b, i, h] = (e / e.sum()) @ v[b, :, h // G]
+                    lse[b, h, i] = m + math.log(e.sum())
+    return out, lse
+
+
+def pin_block_sparse_brute_force(orc):
+    """Random per-(batch, head) masks against the expanded-mask brute force; at
+    scale 0 every row is the mean of the values it sees and lse = ln(count)."""
+    r = _rng(31)
+    for (B, M, N, Hq, Hkv, D, bm, bn) in ((2, 7, 10, 4, 2, 3, 3, 4), (1, 9, 5, 2, 1, 4, 2, 2)):
+        q = r.standard_normal((B, M, Hq, D))
+        k, v = r.standard_normal((B, N, Hkv, D)), r.standard_normal((B, N, Hkv, D))
+        mask = (r.random((B, Hq, -(-M // bm), -(-N // bn))) < 0.6).astype(np.uint8)
+        for causal in (False, True):
+            bias = BIAS_CAUSAL if causal else BIAS_NONE
+            o, l = orc.attention_block_sparse(q, k, v, mask, bm, bn, bias=bias, scale=0.9)
+            ob, lb = brute_force_block_sparse(q, k, v, mask, bm, bn, causal, 0.9)
+            _close(o, ob, tol=1e-10, what="block-sparse brute out")
+            _close(l, lb, tol=1e-10, what="block-sparse brute lse")
+            rows = np.array([[0, M - 1, Hq - 1], [B - 1, 0, 0], [0, M // 2, 1]])
+            orow, lrow = orc.attention_block_sparse(q, k, v, mask, bm, bn, bias=bias, scale=0.9,
+                                                    rows=rows)
+            _close(orow, o[rows[:, 0], rows[:, 1], rows[:, 2]], what="block-sparse rows out")
+            _close(lrow, l[rows[:, 0], rows[:, 2], rows[:, 1]], what="block-sparse rows lse")
+            o0, l0 = orc.attention_block_sparse(q, k, v, mask, bm, bn, bias=bias, scale=0.0)
+            for b in range(B):
+                for h in range(Hq):
+                    for i in range(M):
+                        keys = [j for j in range(N) if mask[b, h, i // bm, j // bn]
+                                and (not causal or j <= i + N - M)]
+                        if not keys:
+                            assert np.isneginf(l0[b, h, i]) and not o0[b, i, h].any()
+                            continue
+                        _close(o0[b, i, h], v[b, keys, h // (Hq // Hkv)].mean(axis=0),
+                               what="block-sparse scale-0 mean")
+                        _close(l0[b, h, i], math.log(len(keys)), what="block-sparse scale-0 lse")
+
+
 PINS = [
     pin_weights_sum_to_one,
     pin_causal_row0_is_v0,
@@ -464,4 +564,6 @@ PINS = [
     pin_bwd_finite_differences,
     pin_bwd_closed_forms,
     pin_bwd_gqa_and_key_shift,
+    pin_block_sparse_reductions,
+    pin_block_sparse_brute_force,
 ]

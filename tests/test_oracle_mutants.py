@@ -36,6 +36,10 @@ MUTANTS = [
     ("bwd_dq_unscaled", "dqi[d] += scale * ds * kj[d];", "dqi[d] += ds * kj[d];", 0),
     ("bwd_dv_from_dp", "dvj[d] += p[j] * doi[d];", "dvj[d] += dp[j] * doi[d];", 0),
     ("bwd_unnormalised", "p[j] /= z;", "p[j] /= 1.0;", 0),
+    ("block_sparse_mask_ignored", "if (keep && !keep[j / block_n]) visible = 0;", "", 0),
+    ("block_sparse_row_block_from_key_size", "+ i / block_m) * nblocks", "+ i / block_n) * nblocks", 0),
+    ("block_sparse_head_ignored", "(((b * Hq + h) * mblocks)", "(((b * Hq) * mblocks)", 0),
+    ("block_sparse_key_block_size_wrong", "!keep[j / block_n]", "!keep[j / (block_n + 1)]", 0),
 ]
 
 
