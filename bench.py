@@ -67,6 +67,24 @@ def prefill_flops(p: synth.Prefill) -> float:
     return 4.0 * p.K * p.Hq * pairs
 
 
+def block_sparse_flops(p: synth.Prefill, mask, block: int = 128) -> float:
+    """4*K per visible (query, key) pair inside the kept blocks (causal pairs
+    only under a causal mask); left-out blocks are not credited."""
+    mb, nb = mask.shape[2], mask.shape[3]
+    off = p.N - p.M
+    pairs = np.zeros((mb, nb))
+    for a in range(mb):
+        rows = np.arange(a * block, min(p.M, (a + 1) * block))
+        for c in range(nb):
+            c0, c1 = c * block, min(p.N, (c + 1) * block)
+            if p.bias == "causal":
+                pairs[a, c] = np.clip(rows + off + 1 - c0, 0, c1 - c0).sum()
+            else:
+                pairs[a, c] = len(rows) * (c1 - c0)
+    m = mask.expand(p.B, p.Hq, mb, nb).to(torch.float64).sum(dim=(0, 1)).numpy()
+    return 4.0 * p.K * float((m * pairs).sum())
+
+
 def decode_bytes(d: synth.Decode) -> float:
     el = 2
     cache = 2.0 * sum(d.kv_lens) * d.Hkv * d.K * el
@@ -276,6 +294,8 @@ def run_ours(args, rank, world, local):
         also["causal_small"] = measure_prefill(mea, synth.causal_small(), dev, stream, tc_peak,
                                                iters=50)
         also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
+        bs_p, bs_mask = synth.block_sparse_noncausal()
+        also["block_sparse"] = measure_block_sparse(mea, bs_p, bs_mask, dev, stream, tc_peak)
         also["bwd_noncausal_m2048"] = measure_backward(mea, synth.noncausal_sweep(2048), dev,
                                                        stream, tc_peak)
         also["bwd_gqa_alibi_causal"] = measure_backward(mea, synth.gqa_alibi_causal(), dev,
@@ -435,6 +455,21 @@ def measure_prefill(mea, p, dev, stream, tc_peak, iters=10):
             "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor"}
 
 
+def measure_block_sparse(mea, p, mask, dev, stream, tc_peak, iters=10):
+    q, k, v = p.q.to(dev), p.k.to(dev), p.v.to(dev)
+    bm = mask.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((p.B, p.Hq, p.M), dtype=torch.float32, device=dev)
+    ms = _time(lambda: mea.mea_fwd_block_sparse(q, k, v, bm, bias=p.bias, scale=p.scale,
+                                                alibi=p.alibi, out=out, lse=lse), stream, iters)
+    f = block_sparse_flops(p, mask)
+    tf = f / (ms * 1e-3) / 1e12
+    kept = float(mask.to(torch.float64).mean())
+    return {"workload": p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
+            "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor",
+            "kept_block_fraction": round(kept, 4)}
+
+
 def measure_backward(mea, p, dev, stream, tc_peak, iters=5):
     """mea_bwd alone (the forward that makes out and lse runs once, untimed).
     Work: five contractions of 2*K FLOP per visible (query, key) pair -- S, dP,
@@ -537,6 +572,7 @@ PROFILE_CASES = {
     "fwd_gqa_alibi_m2048": lambda: ("fwd", synth.gqa_alibi_causal(M=2048, B=2)),
     "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
     "bwd_m2048": lambda: ("bwd", synth.noncausal_sweep(2048)),
+    "block_sparse_m2048": lambda: ("sparse", synth.block_sparse_noncausal(2048)),
     "decode_b16": lambda: ("decode", synth.make_decode(
         "decode_b16", synth.decode_lengths()[:16], 32, 8, 128, "bf16", seed=1005)),
 }
@@ -563,6 +599,12 @@ def run_profile(args):
 
         def fn():
             mea.mea_fwd(q, k, v, bias=w.bias, scale=w.scale, alibi=w.alibi, **kw)
+    elif kind == "sparse":
+        w, mask = w
+        q, k, v, bm = w.q.to(dev), w.k.to(dev), w.v.to(dev), mask.to(dev)
+
+        def fn():
+            mea.mea_fwd_block_sparse(q, k, v, bm, bias=w.bias, scale=w.scale, alibi=w.alibi)
     elif kind == "bwd":
         q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
         dout = synth.randn(tuple(w.q.shape), w.dtype, synth.generator(w.seed + 17)).to(dev)

@@ -180,6 +180,36 @@ int mea_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                        mea_dtype_t dtype, int alibi, float scale, cudaStream_t stream);
 
 /*
+ * mea_fwd_block_sparse -- mea_fwd with whole blocks of the score matrix left
+ * out ("FlashAttention (2022)", section "Cosa mostravano i numeri", which names
+ * the block-sparse variant of the method): the scores of query rows
+ * [128a, 128a + 128) against keys [128c, 128c + 128) of (batch b, query head h)
+ * are dropped (bias -inf) when
+ *     block_mask[b * mask_strides[0] + h * mask_strides[1] + a * ceil(N/128) + c] == 0,
+ * on top of `bias` (MEA_BIAS_NONE or MEA_BIAS_CAUSAL; the block-diagonal kinds
+ * return MEA_ERR_UNSUPPORTED).  Left-out blocks are neither loaded nor
+ * multiplied.  The result is the dense definition with that mask, exact up to
+ * the same rounding as mea_fwd; a row left with no visible key gets out = 0,
+ * lse = -inf.
+ *
+ *   block_mask    DEVICE uint8, [B, Hq, ceil(M/128), ceil(N/128)] with the
+ *                 last two dimensions contiguous; mask_strides (host, elements)
+ *                 step b and h, 0 to share one mask across batches or heads.
+ *   Other arguments as for mea_fwd.  Returns MEA_OK or an error status (a NULL
+ *   mask or negative mask stride: MEA_ERR_INVALID_ARG); never synchronises.
+ */
+int mea_fwd_block_sparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                         int B, int M, int N, int Hq, int Hkv, int K,
+                         const int64_t q_strides[3], const int64_t k_strides[3],
+                         const int64_t v_strides[3], const int64_t o_strides[3],
+                         mea_dtype_t dtype, mea_bias_t bias, const uint8_t* block_mask,
+                         const int64_t mask_strides[2], int alibi, float scale,
+                         cudaStream_t stream);
+
+/* Rows and keys covered by one block-mask entry of mea_fwd_block_sparse (128). */
+int mea_sparse_block_size(void);
+
+/*
  * mea_bwd -- gradients of the attention of mea_fwd ("FlashAttention (2022)",
  * section "Il trucco della softmax che non ha bisogno di vedere tutto": the
  * backward pass recomputes the attention weights from q, k and the forward's

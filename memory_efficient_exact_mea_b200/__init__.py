@@ -8,6 +8,8 @@ is no fallback: importing this package fails loudly if ``libmea.so`` is missing.
 Operations (sources cited in ``include/mea.h``):
   mea_fwd     softmax(Q K^T * scale + bias) V and the per-row log-sum-exp, with
               no / causal / block-diagonal (causal) masks, GQA and ALiBi.
+  mea_fwd_block_sparse  mea_fwd with whole 128x128 score blocks left out by a mask.
+  mea_bwd     dq, dk, dv by recomputing the weights from the forward's lse.
   mea_decode  one query per sequence against a packed, ragged KV cache.
 """
 from __future__ import annotations
@@ -17,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["mea_fwd", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
+__all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
            "read_device_status", "status_string", "MeaError", "BIAS", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
@@ -48,6 +50,11 @@ def _load() -> ctypes.CDLL:
     L.mea_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.mea_decode.restype = i
     L.mea_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, sz, vp]
+    L.mea_fwd_block_sparse.restype = i
+    L.mea_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, i, i,
+                                       vp, vp, i, f, vp]
+    L.mea_sparse_block_size.restype = i
+    L.mea_sparse_block_size.argtypes = []
     L.mea_bwd_workspace_size.restype = sz
     L.mea_bwd_workspace_size.argtypes = [i, i, i, i]
     L.mea_bwd.restype = i
@@ -140,6 +147,45 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
                      _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k), int(bool(alibi)),
                      scale, _stream(stream))
     _check("mea_fwd", rc)
+    return out, lse
+
+
+def mea_fwd_block_sparse(q, k, v, block_mask, bias: str = "none", scale: float | None = None,
+                         alibi: bool = False, out=None, lse=None, return_lse: bool = True,
+                         stream=None):
+    """Block-sparse attention forward.  As ``mea_fwd`` (bias "none" or "causal"),
+    plus ``block_mask``: a uint8 CUDA tensor [B, Hq, ceil(M/128), ceil(N/128)]
+    (size-1 or stride-0 batch/head dimensions broadcast; the last two dimensions
+    contiguous); a zero entry leaves that 128x128 block of scores out."""
+    B, M, Hq, K = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    if q.dtype not in _DTYPE or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype float16 or bfloat16")
+    if tuple(k.shape) != (B, N, Hkv, K) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, N, Hkv, K]")
+    blk = int(lib.mea_sparse_block_size())
+    mb, nb = -(-M // blk), -(-N // blk)
+    if (block_mask.dtype != torch.uint8 or block_mask.dim() != 4 or not block_mask.is_cuda
+            or tuple(block_mask.shape[2:]) != (mb, nb)
+            or block_mask.shape[0] not in (1, B) or block_mask.shape[1] not in (1, Hq)):
+        raise ValueError(f"block_mask must be a uint8 CUDA tensor [B|1, Hq|1, {mb}, {nb}]")
+    if block_mask.stride(3) != 1 or block_mask.stride(2) != nb:
+        raise ValueError("block_mask: the last two dimensions must be contiguous")
+    mst = (ctypes.c_int64 * 2)(block_mask.stride(0) if block_mask.shape[0] > 1 else 0,
+                               block_mask.stride(1) if block_mask.shape[1] > 1 else 0)
+    scale = K ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, M, Hq, K), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, M), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, Hq, M] tensor")
+    rc = lib.mea_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, M, N, Hq,
+                                  Hkv, K, _bmhk_strides(q, "q"), _bmhk_strides(k, "k"),
+                                  _bmhk_strides(v, "v"), _bmhk_strides(out, "out"),
+                                  _DTYPE[q.dtype], BIAS[bias], _ptr(block_mask), mst,
+                                  int(bool(alibi)), scale, _stream(stream))
+    _check("mea_fwd_block_sparse", rc)
     return out, lse
 
 

@@ -110,12 +110,15 @@ const char* mea_status_string(int status) {
 
 int mea_decode_chunk(void) { return mea::kDecodeChunk; }
 
-int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int M,
-            int N, int Hq, int Hkv, int K, const int64_t q_strides[3], const int64_t k_strides[3],
-            const int64_t v_strides[3], const int64_t o_strides[3], mea_dtype_t dtype,
-            mea_bias_t bias, const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
-            int max_seqlen_q, int max_seqlen_k, int alibi, float scale, cudaStream_t stream) {
-  (void)max_seqlen_k;
+// mea_fwd and mea_fwd_block_sparse (block_mask != nullptr: bias none or causal,
+// mask_strides = element strides of the mask for b and h).
+static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                    int M, int N, int Hq, int Hkv, int K, const int64_t q_strides[3],
+                    const int64_t k_strides[3], const int64_t v_strides[3],
+                    const int64_t o_strides[3], mea_dtype_t dtype, mea_bias_t bias,
+                    const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+                    int max_seqlen_q, int alibi, float scale, const uint8_t* block_mask,
+                    const int64_t* mask_strides, cudaStream_t stream) {
   if (B < 0 || M < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return MEA_ERR_INVALID_ARG;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
   if (bias < MEA_BIAS_NONE || bias > MEA_BIAS_BLOCKDIAG_CAUSAL) return MEA_ERR_INVALID_ARG;
@@ -171,12 +174,49 @@ int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   const int rows = packed ? max_seqlen_q : M;
   a.num_mblocks = (rows + mea::kFwdRowsPerCta - 1) / mea::kFwdRowsPerCta;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.block_mask = block_mask;
+  if (block_mask) {
+    a.bm_sb = mask_strides[0];
+    a.bm_sh = mask_strides[1];
+    a.bm_nk = (N + mea::kSparseBlock - 1) / mea::kSparseBlock;
+  }
   L.head_dim = K;
   L.bf16 = bf16;
   L.mask = static_cast<int>(bias);
   L.alibi = alibi != 0;
   if (a.num_mblocks == 0) return MEA_OK;
   return mea::launch_fwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int M,
+            int N, int Hq, int Hkv, int K, const int64_t q_strides[3], const int64_t k_strides[3],
+            const int64_t v_strides[3], const int64_t o_strides[3], mea_dtype_t dtype,
+            mea_bias_t bias, const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+            int max_seqlen_q, int max_seqlen_k, int alibi, float scale, cudaStream_t stream) {
+  (void)max_seqlen_k;
+  return fwd_impl(q, k, v, out, lse, B, M, N, Hq, Hkv, K, q_strides, k_strides, v_strides,
+                  o_strides, dtype, bias, seqstart_q, seqstart_k, num_seqs, max_seqlen_q, alibi,
+                  scale, nullptr, nullptr, stream);
+}
+
+int mea_sparse_block_size(void) { return mea::kSparseBlock; }
+
+int mea_fwd_block_sparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                         int B, int M, int N, int Hq, int Hkv, int K,
+                         const int64_t q_strides[3], const int64_t k_strides[3],
+                         const int64_t v_strides[3], const int64_t o_strides[3],
+                         mea_dtype_t dtype, mea_bias_t bias, const uint8_t* block_mask,
+                         const int64_t mask_strides[2], int alibi, float scale,
+                         cudaStream_t stream) {
+  if (bias != MEA_BIAS_NONE && bias != MEA_BIAS_CAUSAL) {
+    if (bias < MEA_BIAS_NONE || bias > MEA_BIAS_BLOCKDIAG_CAUSAL) return MEA_ERR_INVALID_ARG;
+    return MEA_ERR_UNSUPPORTED;
+  }
+  if (!mask_strides || mask_strides[0] < 0 || mask_strides[1] < 0) return MEA_ERR_INVALID_ARG;
+  if (B > 0 && M > 0 && N > 0 && !block_mask) return MEA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, out, lse, B, M, N, Hq, Hkv, K, q_strides, k_strides, v_strides,
+                  o_strides, dtype, bias, nullptr, nullptr, 0, 0, alibi, scale,
+                  N > 0 ? block_mask : nullptr, mask_strides, stream);
 }
 
 size_t mea_decode_workspace_size(int B, int Hq, int Hkv, int K, int max_kv_len) {

@@ -85,7 +85,10 @@ __device__ long long g_trace[kTraceCtas * kTraceSlots];
   } while (0)
 #endif
 
-template <int D, bool BF16, int MASK, bool ALIBI>
+// SPARSE: a block mask (one byte per 128-query x 128-key block) leaves out
+// whole score tiles ("FlashAttention (2022)", "Cosa mostravano i numeri": the
+// block-sparse variant); a left-out tile is neither loaded nor multiplied.
+template <int D, bool BF16, int MASK, bool ALIBI, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
@@ -168,6 +171,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int nt = max(nt_tile[0], nt_tile[1]);
 
+  // Does query tile t compute key tile j?  Every role walks the key tiles in
+  // the same order and skips those neither query tile needs; the barriers of a
+  // query tile count only the key tiles that tile computes.
+  const uint8_t* mrow0 = nullptr;
+  const uint8_t* mrow1 = nullptr;
+  if constexpr (SPARSE) {
+    const long long base = unit * a.bm_sb + static_cast<long long>(h) * a.bm_sh;
+    mrow0 = a.block_mask + base + static_cast<long long>(2 * mb) * a.bm_nk;
+    mrow1 = mrow0 + a.bm_nk;
+  }
+  auto uses = [&](int t, int j) -> bool {
+    if (j >= nt_tile[t]) return false;
+    if constexpr (SPARSE) return __ldg(t ? mrow1 + j : mrow0 + j) != 0;
+    return true;
+  };
+
   // ---- set-up -----------------------------------------------------------
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -210,6 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                       q0 + m_base + t * kBM, bidx);
       int it = 0;
       for (int j = 0; j < nt; ++j) {
+        if constexpr (SPARSE) {
+          if (!uses(0, j) && !uses(1, j)) continue;
+        }
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % S;
           if (!mbar_wait(&kv_empty[slot], ((it / S) & 1) ^ 1, abort_flag, a.status)) break;
@@ -275,94 +297,124 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Per tile the order is Q.K_j^T, then P.V of the tile the softmax has
       // finished: V_{j-1} in the separate-P layout (Q.K_j^T only needs S_t read out),
       // V_j when P is written over S (Q.K_{j+1}^T must follow P.V_j).
-      const int t = tile, ntt = nt_tile[tile];
-      auto pv_step = [&](int jv) -> bool {
-        const int vs = (2 * jv + 1) % S;
-        if (!mbar_wait(&kv_full[vs], ((2 * jv + 1) / S) & 1, abort_flag, a.status)) return false;
-        MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 2);
-        if (jv < ntt) {
-          if (!mbar_wait(&p_ready[t], jv & 1, abort_flag, a.status)) return false;
-          MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 3);
+      // li counts the key tiles in the ring (both query tiles), c the key tiles
+      // this query tile has computed (its barrier phases).
+      const int t = tile;
+      auto pv_step = [&](int lv, bool used, int cu) -> bool {
+        const int vs = (2 * lv + 1) % S;
+        if (!mbar_wait(&kv_full[vs], ((2 * lv + 1) / S) & 1, abort_flag, a.status)) return false;
+        MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 2);
+        if (used) {
+          if (!mbar_wait(&p_ready[t], cu & 1, abort_flag, a.status)) return false;
+          MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 3);
           tc_fence_after();
-          issue_pv(t, vs, jv > 0);
+          issue_pv(t, vs, cu > 0);
           umma_commit(&o_done[t]);
-          MEA_TRACE_AT(1024 + t * 256 + jv * 8 + 4);
+          MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 4);
         }
         umma_commit(&kv_empty[vs]);
         return true;
       };
       if (kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
-        bool ok = true;
+        bool ok = true, prev_used = false;
+        int li = 0, c = 0, prev_c = 0;
         for (int j = 0; j < nt && ok; ++j) {
-          const int ks = (2 * j) % S;
-          if (!(ok = mbar_wait(&kv_full[ks], ((2 * j) / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + t * 256 + j * 8 + 0);
-          if (j < ntt) {
-            if (j > 0) {  // the softmax has read S_t(j-1) out of TMEM
-              if (!(ok = mbar_wait(&s_free[t], (j - 1) & 1, abort_flag, a.status))) break;
+          const bool used = uses(t, j);
+          if constexpr (SPARSE) {
+            if (!used && !uses(1 - t, j)) continue;
+          } else {
+            li = j;  // dense: every key tile is in the ring and a tile uses a prefix
+            c = j;
+          }
+          const int ks = (2 * li) % S;
+          if (!(ok = mbar_wait(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
+          MEA_TRACE_AT(1024 + t * 256 + li * 8 + 0);
+          if (used) {
+            if (c > 0) {  // the softmax has read the previous S_t out of TMEM
+              if (!(ok = mbar_wait(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
               tc_fence_after();
             }
             issue_qk(t, ks);
             umma_commit(&s_full[t]);
-            MEA_TRACE_AT(1024 + t * 256 + j * 8 + 1);
+            MEA_TRACE_AT(1024 + t * 256 + li * 8 + 1);
           }
           umma_commit(&kv_empty[ks]);
-          if (j >= 1) ok = pv_step(j - 1);
+          if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c);
+          prev_used = used;
+          prev_c = c;
+          c += used ? 1 : 0;
+          ++li;
         }
-        if (ok) pv_step(nt - 1);
+        if constexpr (!SPARSE) li = nt;
+        if (ok && li > 0) pv_step(li - 1, prev_used, prev_c);
       }
       // When P is written over S the chain softmax -> P.V -> Q.K^T of a tile is
       // serial, so one thread (warp 16) issues both tiles in the interleaved
       // order Q0.K_j, P1.V_{j-1}, Q1.K_j, P0.V_j, which keeps the two tiles half a
       // step apart: one tile's softmax overlaps the other tile's MMAs.
       if (!kSepP && tile == 0 && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
-        int it = 0, vslot_prev = 0;
-        bool ok = true;
+        // li: key tiles in the ring; c0, c1: key tiles computed by query tile 0, 1.
+        int it = 0, vslot_prev = 0, li = 0, c0 = 0, c1 = 0, prev_c1 = 0;
+        bool ok = true, prev_u1 = false;
         for (int j = 0; j < nt && ok; ++j) {
+          const bool u0 = uses(0, j), u1 = uses(1, j);
+          if constexpr (SPARSE) {
+            if (!u0 && !u1) continue;
+          } else {  // dense: every key tile is in the ring and each tile uses a prefix
+            li = j;
+            it = 2 * j;
+            c0 = j;
+            c1 = j;
+          }
           const int kslot = it % S;
           if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + j * 16 + 0);
+          MEA_TRACE_AT(1024 + li * 16 + 0);
           ++it;
-          if (j < nt_tile[0]) {
+          if (u0) {
             issue_qk(0, kslot);
-            MEA_TRACE_AT(1024 + j * 16 + 1);
+            MEA_TRACE_AT(1024 + li * 16 + 1);
             umma_commit(&s_full[0]);
           }
-          if (j >= 1) {
-            if (j - 1 < nt_tile[1]) {
-              if (!(ok = mbar_wait(&p_ready[1], (j - 1) & 1, abort_flag, a.status))) break;
-              MEA_TRACE_AT(1024 + j * 16 + 2);
+          if (li >= 1) {
+            if (prev_u1) {
+              if (!(ok = mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status))) break;
+              MEA_TRACE_AT(1024 + li * 16 + 2);
               tc_fence_after();
-              issue_pv(1, vslot_prev, j - 1 > 0);
+              issue_pv(1, vslot_prev, prev_c1 > 0);
               umma_commit(&o_done[1]);
             }
             umma_commit(&kv_empty[vslot_prev]);
           }
-          if (j < nt_tile[1]) {
+          if (u1) {
             issue_qk(1, kslot);
-            MEA_TRACE_AT(1024 + j * 16 + 3);
+            MEA_TRACE_AT(1024 + li * 16 + 3);
             umma_commit(&s_full[1]);
           }
           umma_commit(&kv_empty[kslot]);
           const int vslot = it % S;
           if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + j * 16 + 4);
+          MEA_TRACE_AT(1024 + li * 16 + 4);
           ++it;
-          if (j < nt_tile[0]) {
-            if (!(ok = mbar_wait(&p_ready[0], j & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + j * 16 + 5);
+          if (u0) {
+            if (!(ok = mbar_wait(&p_ready[0], c0 & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + li * 16 + 5);
             tc_fence_after();
-            issue_pv(0, vslot, j > 0);
-            MEA_TRACE_AT(1024 + j * 16 + 6);
+            issue_pv(0, vslot, c0 > 0);
+            MEA_TRACE_AT(1024 + li * 16 + 6);
             umma_commit(&o_done[0]);
+            ++c0;
           }
           vslot_prev = vslot;
+          prev_u1 = u1;
+          prev_c1 = c1;
+          c1 += u1 ? 1 : 0;
+          ++li;
         }
-        if (ok) {
-          const int j = nt - 1;
-          if (j < nt_tile[1] && mbar_wait(&p_ready[1], j & 1, abort_flag, a.status)) {
+        if constexpr (!SPARSE) li = nt;
+        if (ok && li > 0) {
+          if (prev_u1 && mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status)) {
             tc_fence_after();
-            issue_pv(1, vslot_prev, j > 0);
+            issue_pv(1, vslot_prev, prev_c1 > 0);
             umma_commit(&o_done[1]);
           }
           umma_commit(&kv_empty[vslot_prev]);
@@ -405,8 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l_sum = 0.f;        // this thread's part of the running sum of 2^(x - m_ref)
     bool ok = true;
 
+    int nc = 0;  // key tiles this query tile has computed (its barrier phases)
     for (int j = 0; j < ntt; ++j) {
-      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag, a.status))) break;
+      if constexpr (SPARSE) {
+        if (!uses(t, j)) continue;
+      } else {
+        nc = j;  // dense: every key tile up to ntt is computed
+      }
+      if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
       tc_fence_after();
       uint32_t sr[2][32];
@@ -454,10 +512,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (!ALIBI) pmax = (pmax == neg_inf()) ? pmax : pmax * a.scale_log2;
 
       // ---- exchange with the other half of the row -----------------------------
-      float* xm = xmax + ((t * 2 + (j & 1)) * 2) * kBM;
+      float* xm = xmax + ((t * 2 + (nc & 1)) * 2) * kBM;
       xm[half * kBM + row] = pmax;
       mbar_arrive(pbar);
-      if (!(ok = mbar_wait_warp(pbar, j & 1, abort_flag, a.status))) break;
+      if (!(ok = mbar_wait_warp(pbar, nc & 1, abort_flag, a.status))) break;
       const float tmax = fmaxf(pmax, xm[(1 - half) * kBM + row]);
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
       float m_use = m_ref;
@@ -485,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
       if constexpr (kSepP) {  // P_t is still being read by P.V of the previous tile
-        if (j > 0 && !(ok = mbar_wait_warp(&o_done[t], (j - 1) & 1, abort_flag, a.status))) break;
+        if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
         tc_fence_after();
       }
       // Store P as 16-bit pairs over each 32-key chunk's own S columns (keys
@@ -514,9 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // Rescale this thread's half of the output accumulator when the row's
       // reference max moved.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (nc > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
-        if (!(ok = mbar_wait_warp(&o_done[t], (j - 1) & 1, abort_flag, a.status))) break;
+        if (!(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -532,15 +590,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_ready[t]);
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
+      ++nc;
     }
 
     // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
-    if (ok && ntt > 0) ok = mbar_wait_warp(&o_done[t], (ntt - 1) & 1, abort_flag, a.status);
+    if constexpr (!SPARSE) nc = ntt;
+    if (ok && nc > 0) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
     if (ok) {
       // Row sum = both halves' parts (same reference max).
       xsum[(t * 2 + half) * kBM + row] = l_sum;
       mbar_arrive(pbar);
-      ok = mbar_wait_warp(pbar, ntt & 1, abort_flag, a.status);
+      ok = mbar_wait_warp(pbar, nc & 1, abort_flag, a.status);
     }
     if (ok) {
       const float l_tot = l_sum + xsum[(t * 2 + 1 - half) * kBM + row];
@@ -553,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
-        if (ntt > 0) {
+        if (nc > 0) {
           tmem_ld32(o_addr + c * 32, o);
           tmem_ld_wait(o);
         } else {
@@ -587,9 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool BF16, int MASK, bool ALIBI>
+template <int D, bool BF16, int MASK, bool ALIBI, bool SPARSE = false>
 cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
-  auto kern = fwd_kernel<D, BF16, MASK, ALIBI>;
+  auto kern = fwd_kernel<D, BF16, MASK, ALIBI, SPARSE>;
   const int smem = Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -603,6 +663,15 @@ cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
 
 template <int D, bool BF16>
 cudaError_t dispatch_mask(const FwdLaunch& L, cudaStream_t s) {
+  if (L.args.block_mask != nullptr) {  // block-sparse: no mask or causal only
+    switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
+      case 0: return launch_t<D, BF16, 0, false, true>(L, s);
+      case 1: return launch_t<D, BF16, 0, true, true>(L, s);
+      case 2: return launch_t<D, BF16, 1, false, true>(L, s);
+      case 3: return launch_t<D, BF16, 1, true, true>(L, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
     case 0: return launch_t<D, BF16, 0, false>(L, s);
     case 1: return launch_t<D, BF16, 0, true>(L, s);

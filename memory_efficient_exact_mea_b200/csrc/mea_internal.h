@@ -22,7 +22,14 @@ struct FwdArgs {
   int num_units;    // B for dense batches, num_seqs for packed ones
   int num_mblocks;  // ceil(max query rows per unit / kFwdRowsPerCta)
   float scale_log2; // scale * log2(e)
+  // Block-sparse only (nullptr otherwise): byte [b * bm_sb + h * bm_sh +
+  // (query row / 128) * bm_nk + key / 128], zero = block left out.
+  const uint8_t* block_mask;
+  long long bm_sb, bm_sh;
+  int bm_nk;        // ceil(N / 128)
 };
+
+constexpr int kSparseBlock = 128;  // rows and keys per block-mask entry
 
 struct FwdLaunch {
   CUtensorMap tmQ, tmK, tmV;

@@ -184,3 +184,25 @@ def decode_step() -> Decode:
     """Decode: B=64, cached lengths U[512, 8192], Hq=32, Hkv=8, K=128, bf16 cache."""
     return make_decode("decode_b64_kv512-8192_hq32_hkv8_k128_bf16", decode_lengths(), 32, 8, 128,
                        "bf16", seed=1005)
+
+
+def block_mask(B: int, Hq: int, M: int, N: int, block: int, density: float, seed: int,
+               keep_diagonal: bool = False) -> torch.Tensor:
+    """uint8 [B, Hq, ceil(M/block), ceil(N/block)]: each block kept (1) with
+    probability `density` (independent uniform draws); with keep_diagonal the
+    blocks (i, i) are always kept."""
+    mb, nb = -(-M // block), -(-N // block)
+    u = torch.rand((B, Hq, mb, nb), generator=generator(seed), dtype=torch.float32)
+    m = (u < density).to(torch.uint8)
+    if keep_diagonal:
+        d = torch.arange(min(mb, nb))
+        m[:, :, d, d] = 1
+    return m
+
+
+def block_sparse_noncausal(M: int = 4096) -> tuple[Prefill, torch.Tensor]:
+    """Block-sparse non-causal: the sweep's B=8, H=16, K=64, fp16 at M=N, with 128x128
+    blocks kept with probability 1/2 per (batch, head), diagonal blocks always kept."""
+    p = make_prefill(f"block_sparse_b8_h16_k64_f16_m{M}_d50", 8, M, M, 16, 16, 64, "f16", "none",
+                     seed=1006)
+    return p, block_mask(8, 16, M, M, 128, 0.5, seed=1007, keep_diagonal=True)

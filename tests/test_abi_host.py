@@ -179,3 +179,23 @@ def test_bwd_rejects_bad_arguments(lib):
     assert _bwd(lib, ws=512 + 16) == WORKSPACE             # 256-byte alignment
     assert _bwd(lib, B=0) == 0
     assert _bwd(lib, M=0, N=0) == 0
+
+
+def test_block_sparse_rejects_bad_arguments(lib):
+    INVALID, UNSUPPORTED = -1, -2
+    vp = ctypes.c_void_p
+
+    def call(bias=0, mask=16, ms=(0, 0), K=64, scale=0.1):
+        s = I64x3(1024, 64 * 4, 64)
+        mst = (ctypes.c_int64 * 2)(*ms) if ms is not None else None
+        return lib.mea_fwd_block_sparse(vp(16), vp(16), vp(16), vp(16), None, 1, 128, 128, 4, 4,
+                                        K, s, s, s, s, 0, bias, vp(mask), mst, 0,
+                                        ctypes.c_float(scale), None)
+    assert lib.mea_sparse_block_size() == 128
+    assert call(bias=2) == UNSUPPORTED
+    assert call(bias=3) == UNSUPPORTED
+    assert call(bias=7) == INVALID
+    assert call(mask=None) == INVALID
+    assert call(ms=(-1, 0)) == INVALID
+    assert call(ms=None) == INVALID
+    assert call(K=96) == UNSUPPORTED
