@@ -75,6 +75,9 @@ class Oracle:
         lib.oracle_attention_block_sparse.argtypes = [_c_double_p] * 3 + [ctypes.c_int] * 7 + [
             _c_uint8_p, ctypes.c_int, ctypes.c_int, _c_double_p, ctypes.c_double, _c_int64_p,
             ctypes.c_int64, _c_double_p, _c_double_p]
+        lib.oracle_prefill_chunk.restype = ctypes.c_int
+        lib.oracle_prefill_chunk.argtypes = [_c_double_p] * 5 + [_c_int32_p, _c_int32_p] + [
+            ctypes.c_int] * 7 + [_c_double_p, ctypes.c_double, _c_double_p, _c_double_p]
         lib.oracle_decode.restype = ctypes.c_int
         lib.oracle_decode.argtypes = [_c_double_p, _c_double_p, _c_double_p, _c_int32_p,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -210,6 +213,33 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_attention_block_sparse rejected its arguments")
         return out, lse
+
+    def prefill_chunk(self, q, k_new, v_new, k_cache, v_cache, cache_len, q_len=None,
+                      causal=True, scale=None, alibi=None):
+        """One prefill chunk against a cache.  q [B,M,Hq,D], k_new/v_new [B,M,Hkv,D],
+        caches [B,cap,Hkv,D], cache_len [B] (rows already cached), q_len [B] or None
+        (= M) -> (out [B,M,Hq,D], lse [B,Hq,M], k_cache', v_cache').  Rows i >= q_len[b]
+        of out are 0 and of lse are nan (not computed)."""
+        q, kn, vn = _f64(q), _f64(k_new), _f64(v_new)
+        kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
+        B, M, Hq, D = q.shape
+        cap, Hkv = kc.shape[1], kc.shape[2]
+        assert kn.shape == (B, M, Hkv, D) and vn.shape == kn.shape
+        assert kc.shape == (B, cap, Hkv, D) and vc.shape == kc.shape
+        scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+        cl = _i32(cache_len)
+        ql = _i32(q_len)
+        slopes = self._slopes(alibi, Hq)
+        out = np.zeros((B, M, Hq, D), dtype=np.float64)
+        lse = np.full((B, Hq, M), np.nan, dtype=np.float64)
+        rc = self.lib.oracle_prefill_chunk(
+            _ptr(q, _c_double_p), _ptr(kn, _c_double_p), _ptr(vn, _c_double_p),
+            _ptr(kc, _c_double_p), _ptr(vc, _c_double_p), _ptr(cl, _c_int32_p),
+            _ptr(ql, _c_int32_p), B, M, cap, Hq, Hkv, D, int(bool(causal)),
+            _ptr(slopes, _c_double_p), scale, _ptr(out, _c_double_p), _ptr(lse, _c_double_p))
+        if rc != 0:
+            raise ValueError("oracle_prefill_chunk rejected its arguments")
+        return out, lse, kc, vc
 
     # -- decode --------------------------------------------------------------
     def decode(self, q, k_cache, v_cache, kv_seqstart, scale=None, alibi=None):

@@ -423,3 +423,96 @@ int oracle_attention_bwd(const double* q, const double* k, const double* v, cons
     }
     return failed ? -1 : 0;
 }
+
+/*
+ * One chunk of prefill against a KV cache ("Transformer : comprendre
+ * l'entrainement et l'inference", sections "Pre-remplissage et decodage" and
+ * "Un cache KV simple": the keys and values of the new tokens are concatenated
+ * after the cached ones, and the new queries attend to the whole result under
+ * tril(ones(seq_len, total_len), diagonal=past_len)).
+ * For sequence b with past = cache_len[b] cached rows and n = q_len[b] new rows
+ * (q_len NULL: n = M for every sequence):
+ *   1. append: k_cache[b, past + r] = k_new[b, r], v likewise, for r < n;
+ *   2. for query row i < n (position past + i) and query head h: attention over
+ *      cache rows j < past + n, causal: visible iff j <= past + i; ALiBi bias
+ *      -slope_h * |past + i - j|; weights and lse as in oracle_attention.
+ * Rows i >= n of out and lse are left as they are.
+ *   q, out [B, M, Hq, D]   k_new, v_new [B, M, Hkv, D]   lse [B, Hq, M]
+ *   k_cache, v_cache [B, cap, Hkv, D] (updated in place)
+ * Returns -1 if past < 0, n outside [0, M] or past + n > cap.
+ */
+int oracle_prefill_chunk(const double* q, const double* k_new, const double* v_new,
+                         double* k_cache, double* v_cache, const int32_t* cache_len,
+                         const int32_t* q_len, int B, int M, int cap, int Hq, int Hkv, int D,
+                         int causal, const double* slopes, double scale, double* out,
+                         double* lse) {
+    if (B < 0 || M < 0 || cap < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    if (!cache_len) return -1;
+    for (int b = 0; b < B; ++b) {
+        const int64_t past = cache_len[b], n = q_len ? q_len[b] : M;
+        if (past < 0 || n < 0 || n > M || past + n > cap) return -1;
+    }
+    const int group = Hq / Hkv;
+    /* 1. the append */
+    for (int b = 0; b < B; ++b) {
+        const int64_t past = cache_len[b], n = q_len ? q_len[b] : M;
+        for (int64_t r = 0; r < n; ++r)
+            for (int kvh = 0; kvh < Hkv; ++kvh)
+                for (int d = 0; d < D; ++d) {
+                    const int64_t src = ((b * (int64_t)M + r) * Hkv + kvh) * D + d;
+                    const int64_t dst = ((b * (int64_t)cap + past + r) * Hkv + kvh) * D + d;
+                    k_cache[dst] = k_new[src];
+                    v_cache[dst] = v_new[src];
+                }
+    }
+    /* 2. attention of the chunk's queries over the extended cache */
+    int failed = 0;
+#pragma omp parallel
+    {
+        double* w = (double*)malloc(sizeof(double) * (cap > 0 ? (size_t)cap : 1));
+        if (!w) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t task = 0; task < (int64_t)B * Hq * M; ++task) {
+                const int b = (int)(task / ((int64_t)Hq * M));
+                const int h = (int)((task / M) % Hq);
+                const int64_t i = task % M;
+                const int64_t past = cache_len[b], n = q_len ? q_len[b] : M;
+                if (i >= n) continue;
+                const int kvh = h / group;
+                const int64_t total = past + n, pos_i = past + i;
+                const double* qi = q + ((b * (int64_t)M + i) * Hq + h) * D;
+                double* o = out + ((b * (int64_t)M + i) * Hq + h) * D;
+                double mx = -INFINITY;
+                for (int64_t j = 0; j < total; ++j) {
+                    if (causal && j > pos_i) { w[j] = -INFINITY; continue; }
+                    const double* kj = k_cache + ((b * (int64_t)cap + j) * Hkv + kvh) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+                    double s = scale * dot;
+                    if (slopes) s -= slopes[h] * fabs((double)(pos_i - j));
+                    w[j] = s;
+                    if (s > mx) mx = s;
+                }
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                double* l = lse + ((int64_t)b * Hq + h) * M + i;
+                if (mx == -INFINITY) { *l = -INFINITY; continue; }
+                double z = 0.0;
+                for (int64_t j = 0; j < total; ++j) {
+                    w[j] = (w[j] == -INFINITY) ? 0.0 : exp(w[j] - mx);
+                    z += w[j];
+                }
+                for (int64_t j = 0; j < total; ++j) {
+                    if (w[j] == 0.0) continue;
+                    const double* vj = v_cache + ((b * (int64_t)cap + j) * Hkv + kvh) * D;
+                    for (int d = 0; d < D; ++d) o[d] += (w[j] / z) * vj[d];
+                }
+                *l = mx + log(z);
+            }
+            free(w);
+        }
+    }
+    return failed ? -1 : 0;
+}

@@ -17,6 +17,9 @@ Passages (page title, section):
             of a row sum to one; the result is exact.
   [sparse]  "FlashAttention (2022)", "Cosa mostravano i numeri": the block-sparse
             variant leaves out whole blocks of the score matrix; exact otherwise.
+  [chunk]   "Transformer : comprendre ...", "Pre-remplissage et decodage" and "Un cache
+            KV simple": new keys/values are concatenated after the cached ones and the
+            new queries attend under tril(diagonal=past_len).
 """
 from __future__ import annotations
 
@@ -546,6 +549,80 @@ def pin_block_sparse_brute_force(orc):
                         _close(l0[b, h, i], math.log(len(keys)), what="block-sparse scale-0 lse")
 
 
+# ---------------------------------------------------------------------------
+# [chunk] prefill in chunks against a cache.
+# ---------------------------------------------------------------------------
+def pin_chunks_equal_full_prefill(orc):
+    """Causal prefill of a sequence in two chunks (the second against the cache the
+    first one filled) gives the rows of one causal prefill of the whole sequence,
+    and leaves the whole sequence's keys/values in the cache (GQA, ALiBi, two
+    sequences of different lengths split at different points)."""
+    r = _rng(40)
+    B, Hq, Hkv, D, cap = 2, 4, 2, 3, 12
+    lens, split = [9, 6], [4, 5]
+    q_full = r.standard_normal((B, 9, Hq, D))
+    k_full, v_full = r.standard_normal((B, 9, Hkv, D)), r.standard_normal((B, 9, Hkv, D))
+    kc = np.full((B, cap, Hkv, D), 7.0)
+    vc = np.full((B, cap, Hkv, D), -7.0)
+    M1, M2 = 5, 5
+    q1, k1, v1 = (np.zeros((B, M1) + x.shape[2:]) for x in (q_full, k_full, v_full))
+    q2, k2, v2 = (np.zeros((B, M2) + x.shape[2:]) for x in (q_full, k_full, v_full))
+    for b in range(B):
+        a, n = split[b], lens[b]
+        q1[b, :a], k1[b, :a], v1[b, :a] = q_full[b, :a], k_full[b, :a], v_full[b, :a]
+        q2[b, :n - a], k2[b, :n - a], v2[b, :n - a] = (q_full[b, a:n], k_full[b, a:n],
+                                                       v_full[b, a:n])
+    o1, l1, kc, vc = orc.prefill_chunk(q1, k1, v1, kc, vc, [0, 0], q_len=split, alibi=True)
+    past = split
+    o2, l2, kc, vc = orc.prefill_chunk(q2, k2, v2, kc, vc, past,
+                                       q_len=[lens[b] - split[b] for b in range(B)], alibi=True)
+    for b in range(B):
+        n, a = lens[b], split[b]
+        of, lf = orc.attention(q_full[b:b + 1, :n], k_full[b:b + 1, :n], v_full[b:b + 1, :n],
+                               bias=BIAS_CAUSAL, alibi=True)
+        _close(o1[b, :a], of[0, :a], what="chunk 1 out")
+        _close(l1[b, :, :a], lf[0, :, :a], what="chunk 1 lse")
+        _close(o2[b, :n - a], of[0, a:n], what="chunk 2 out")
+        _close(l2[b, :, :n - a], lf[0, :, a:n], what="chunk 2 lse")
+        _close(kc[b, :n], k_full[b, :n], what="cache keys")
+        _close(vc[b, :n], v_full[b, :n], what="cache values")
+        assert np.all(kc[b, n:] == 7.0) and np.all(vc[b, n:] == -7.0), "rows past the end"
+        assert not o2[b, n - a:].any() and np.isnan(l2[b, :, n - a:]).all(), "padding rows"
+
+
+def pin_chunk_of_one_is_decode(orc):
+    """A one-row chunk is a decode step against the cache it extends."""
+    r = _rng(41)
+    B, Hq, Hkv, D, cap = 3, 4, 2, 5, 10
+    past = [0, 4, 9]
+    kc, vc = r.standard_normal((B, cap, Hkv, D)), r.standard_normal((B, cap, Hkv, D))
+    q, kn, vn = (r.standard_normal((B, 1, H, D)) for H in (Hq, Hkv, Hkv))
+    for alibi in (False, True):
+        o, l, kc2, vc2 = orc.prefill_chunk(q, kn, vn, kc, vc, past, causal=True, alibi=alibi)
+        packed_k = np.concatenate([kc2[b, :past[b] + 1] for b in range(B)])
+        packed_v = np.concatenate([vc2[b, :past[b] + 1] for b in range(B)])
+        od, ld = orc.decode(q[:, 0], packed_k, packed_v, _offsets([p + 1 for p in past]),
+                            alibi=alibi)
+        _close(o[:, 0], od, what="one-row chunk = decode out")
+        _close(l[:, :, 0], ld, what="one-row chunk = decode lse")
+
+
+def pin_noncausal_chunk(orc):
+    """Without the causal mask a chunk's queries see every cached and new key:
+    the plain attention over the concatenation (positions past + i for ALiBi)."""
+    r = _rng(42)
+    B, M, Hq, Hkv, D, cap = 1, 4, 2, 1, 3, 9
+    past = 5
+    kc, vc = r.standard_normal((B, cap, Hkv, D)), r.standard_normal((B, cap, Hkv, D))
+    q, kn, vn = (r.standard_normal((B, M, H, D)) for H in (Hq, Hkv, Hkv))
+    o, l, _, _ = orc.prefill_chunk(q, kn, vn, kc, vc, [past], causal=False, alibi=True)
+    k_all = np.concatenate([kc[:, :past], kn], axis=1)
+    v_all = np.concatenate([vc[:, :past], vn], axis=1)
+    od, ld = orc.attention(q, k_all, v_all, bias=BIAS_NONE, alibi=True)
+    _close(o, od, what="non-causal chunk out")
+    _close(l, ld, what="non-causal chunk lse")
+
+
 PINS = [
     pin_weights_sum_to_one,
     pin_causal_row0_is_v0,
@@ -566,4 +643,7 @@ PINS = [
     pin_bwd_gqa_and_key_shift,
     pin_block_sparse_reductions,
     pin_block_sparse_brute_force,
+    pin_chunks_equal_full_prefill,
+    pin_chunk_of_one_is_decode,
+    pin_noncausal_chunk,
 ]

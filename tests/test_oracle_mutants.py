@@ -39,6 +39,11 @@ MUTANTS = [
     ("block_sparse_mask_ignored", "if (keep && !keep[j / block_n]) visible = 0;", "", 0),
     ("block_sparse_row_block_from_key_size", "+ i / block_m) * nblocks", "+ i / block_n) * nblocks", 0),
     ("block_sparse_head_ignored", "(((b * Hq + h) * mblocks)", "(((b * Hq) * mblocks)", 0),
+    ("chunk_append_at_start", "(b * (int64_t)cap + past + r)", "(b * (int64_t)cap + r)", 0),
+    ("chunk_causal_without_past", "if (causal && j > pos_i)", "if (causal && j > i)", 0),
+    ("chunk_alibi_without_past", "fabs((double)(pos_i - j))", "fabs((double)(i - j))", 0),
+    ("chunk_new_keys_missing", "total = past + n, pos_i", "total = past, pos_i", 0),
+    ("chunk_value_from_key", "const double* vj = v_cache +", "const double* vj = k_cache +", 1),
     ("block_sparse_key_block_size_wrong", "!keep[j / block_n]", "!keep[j / (block_n + 1)]", 0),
 ]
 
