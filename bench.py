@@ -85,6 +85,15 @@ def block_sparse_flops(p: synth.Prefill, mask, block: int = 128) -> float:
     return 4.0 * p.K * float((m * pairs).sum())
 
 
+def chunk_flops(c: synth.Chunk) -> float:
+    """4*K*Hq per visible pair: every cached row, plus the chunk's own rows up to
+    the diagonal (all of them without the causal mask)."""
+    pairs = 0
+    for p, n in zip(c.past, c.q_lens):
+        pairs += p * n + (n * (n + 1) // 2 if c.causal else n * n)
+    return 4.0 * c.K * c.Hq * pairs
+
+
 def decode_bytes(d: synth.Decode) -> float:
     el = 2
     cache = 2.0 * sum(d.kv_lens) * d.Hkv * d.K * el
@@ -294,6 +303,7 @@ def run_ours(args, rank, world, local):
         also["causal_small"] = measure_prefill(mea, synth.causal_small(), dev, stream, tc_peak,
                                                iters=50)
         also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
+        also["chunk_prefill"] = measure_chunk(mea, synth.chunk_prefill(), dev, stream, tc_peak)
         bs_p, bs_mask = synth.block_sparse_noncausal()
         also["block_sparse"] = measure_block_sparse(mea, bs_p, bs_mask, dev, stream, tc_peak)
         also["bwd_noncausal_m2048"] = measure_backward(mea, synth.noncausal_sweep(2048), dev,
@@ -470,6 +480,24 @@ def measure_block_sparse(mea, p, mask, dev, stream, tc_peak, iters=10):
             "kept_block_fraction": round(kept, 4)}
 
 
+def measure_chunk(mea, c: synth.Chunk, dev, stream, tc_peak, iters=10):
+    """mea_prefill_chunk: attention of the chunk plus the fused append, timed
+    together (the same chunk re-appended each iteration)."""
+    q, kn, vn = c.q.to(dev), c.k_new.to(dev), c.v_new.to(dev)
+    kc, vc = c.k_cache.to(dev), c.v_cache.to(dev)
+    cl = torch.tensor(c.past, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((c.B, c.Hq, c.M), dtype=torch.float32, device=dev)
+    ms = _time(lambda: mea.mea_prefill_chunk(q, kn, vn, kc, vc, cl, causal=c.causal,
+                                             scale=c.scale, alibi=c.alibi, out=out, lse=lse),
+               stream, iters)
+    f = chunk_flops(c)
+    tf = f / (ms * 1e-3) / 1e12
+    return {"workload": c.name, "ms": round(ms, 4), "tflops": round(tf, 1),
+            "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor",
+            "note": "includes the append of 512 rows x 8 kv heads per sequence"}
+
+
 def measure_backward(mea, p, dev, stream, tc_peak, iters=5):
     """mea_bwd alone (the forward that makes out and lse runs once, untimed).
     Work: five contractions of 2*K FLOP per visible (query, key) pair -- S, dP,
@@ -573,6 +601,7 @@ PROFILE_CASES = {
     "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
     "bwd_m2048": lambda: ("bwd", synth.noncausal_sweep(2048)),
     "block_sparse_m2048": lambda: ("sparse", synth.block_sparse_noncausal(2048)),
+    "chunk_prefill": lambda: ("chunk", synth.chunk_prefill()),
     "decode_b16": lambda: ("decode", synth.make_decode(
         "decode_b16", synth.decode_lengths()[:16], 32, 8, 128, "bf16", seed=1005)),
 }
@@ -605,6 +634,13 @@ def run_profile(args):
 
         def fn():
             mea.mea_fwd_block_sparse(q, k, v, bm, bias=w.bias, scale=w.scale, alibi=w.alibi)
+    elif kind == "chunk":
+        q, kn, vn = w.q.to(dev), w.k_new.to(dev), w.v_new.to(dev)
+        kc, vc = w.k_cache.to(dev), w.v_cache.to(dev)
+        cl = torch.tensor(w.past, dtype=torch.int32, device=dev)
+
+        def fn():
+            mea.mea_prefill_chunk(q, kn, vn, kc, vc, cl, causal=w.causal, scale=w.scale)
     elif kind == "bwd":
         q, k, v = w.q.to(dev), w.k.to(dev), w.v.to(dev)
         dout = synth.randn(tuple(w.q.shape), w.dtype, synth.generator(w.seed + 17)).to(dev)

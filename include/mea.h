@@ -210,6 +210,44 @@ int mea_fwd_block_sparse(const void* q, const void* k, const void* v, void* out,
 int mea_sparse_block_size(void);
 
 /*
+ * mea_prefill_chunk -- one chunk of prefill against a KV cache, with the cache
+ * append fused into the attention launch ("Transformer : comprendre
+ * l'entrainement et l'inference", sections "Pre-remplissage et decodage" and
+ * "Un cache KV simple": the chunk's keys and values go after the cached ones,
+ * and its queries attend to all of them under tril(diagonal=past_len)).
+ * For sequence b with past = cache_seqlens[b] and n = q_seqlens[b] (M if
+ * q_seqlens is NULL):
+ *   1. k_cache[b, past + r] = k_new[b, r] and v_cache likewise, r < n;
+ *   2. out[b, i], lse[b, :, i] for i < n: attention of q[b, i] (position
+ *      past + i) over cache rows [0, past + n); causal: keys j <= past + i;
+ *      ALiBi distance |past + i - j|; GQA as in mea_fwd.
+ *
+ *   q, out          [B, M, Hq, K]           element strides (b, m, h), K contiguous
+ *   k_new, v_new    [B, M, Hkv, K]          the chunk's keys/values (rows >= n unused)
+ *   k_cache, v_cache [B, cache_rows, Hkv, K] updated in place (rows [past, past+n))
+ *   cache_seqlens   DEVICE int32 [B]        rows cached before the call (not updated:
+ *                                           the caller adds n afterwards)
+ *   q_seqlens       DEVICE int32 [B] or NULL real rows of each chunk (<= M)
+ *   lse             [B, Hq, M] fp32 natural log, or NULL
+ * Rows i >= n of out and lse are not written.  The launch reads cache rows
+ * [0, past) only (the new rows come from k_new), so cache rows from past on may
+ * hold anything; rows outside [past, past + n) are not written.  A sequence with past < 0, n
+ * outside [0, M] or past + n > cache_rows is skipped and records
+ * MEA_ERR_INVALID_ARG in the device status word.  cache_rows must be >= 1.
+ * The caches must not overlap q, k_new, v_new or out.  Other conventions as
+ * for mea_fwd (causal is 0 or 1).  Returns MEA_OK or an error status; never
+ * synchronises.
+ */
+int mea_prefill_chunk(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                      void* v_cache, const int32_t* cache_seqlens, const int32_t* q_seqlens,
+                      void* out, float* lse, int B, int M, int cache_rows, int Hq, int Hkv,
+                      int K, const int64_t q_strides[3], const int64_t kn_strides[3],
+                      const int64_t vn_strides[3], const int64_t kc_strides[3],
+                      const int64_t vc_strides[3], const int64_t o_strides[3],
+                      mea_dtype_t dtype, int causal, int alibi, float scale,
+                      cudaStream_t stream);
+
+/*
  * mea_bwd -- gradients of the attention of mea_fwd ("FlashAttention (2022)",
  * section "Il trucco della softmax che non ha bisogno di vedere tutto": the
  * backward pass recomputes the attention weights from q, k and the forward's

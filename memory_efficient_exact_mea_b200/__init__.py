@@ -9,6 +9,7 @@ Operations (sources cited in ``include/mea.h``):
   mea_fwd     softmax(Q K^T * scale + bias) V and the per-row log-sum-exp, with
               no / causal / block-diagonal (causal) masks, GQA and ALiBi.
   mea_fwd_block_sparse  mea_fwd with whole 128x128 score blocks left out by a mask.
+  mea_prefill_chunk  a chunk of new queries against a KV cache, appending its keys/values.
   mea_bwd     dq, dk, dv by recomputing the weights from the forward's lse.
   mea_decode  one query per sequence against a packed, ragged KV cache.
 """
@@ -19,7 +20,7 @@ import os
 
 import torch
 
-__all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
+__all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_prefill_chunk", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
            "read_device_status", "status_string", "MeaError", "BIAS", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
@@ -53,6 +54,8 @@ def _load() -> ctypes.CDLL:
     L.mea_fwd_block_sparse.restype = i
     L.mea_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, i, i,
                                        vp, vp, i, f, vp]
+    L.mea_prefill_chunk.restype = i
+    L.mea_prefill_chunk.argtypes = [vp] * 9 + [i] * 6 + [vp] * 6 + [i, i, i, f, vp]
     L.mea_sparse_block_size.restype = i
     L.mea_sparse_block_size.argtypes = []
     L.mea_bwd_workspace_size.restype = sz
@@ -186,6 +189,47 @@ def mea_fwd_block_sparse(q, k, v, block_mask, bias: str = "none", scale: float |
                                   _DTYPE[q.dtype], BIAS[bias], _ptr(block_mask), mst,
                                   int(bool(alibi)), scale, _stream(stream))
     _check("mea_fwd_block_sparse", rc)
+    return out, lse
+
+
+def mea_prefill_chunk(q, k_new, v_new, k_cache, v_cache, cache_seqlens, q_seqlens=None,
+                      causal: bool = True, scale: float | None = None, alibi: bool = False,
+                      out=None, lse=None, return_lse: bool = True, stream=None):
+    """One prefill chunk against a KV cache, with the append fused in.
+
+    q [B,M,Hq,K], k_new/v_new [B,M,Hkv,K], k_cache/v_cache [B,cap,Hkv,K] (updated
+    in place: rows cache_seqlens[b] .. + q_seqlens[b] receive the chunk's keys and
+    values), cache_seqlens / q_seqlens int32 CUDA [B] (q_seqlens None: every
+    sequence has M new rows).  Returns (out [B,M,Hq,K], lse [B,Hq,M] or None);
+    rows past q_seqlens[b] are not written.  The caller advances cache_seqlens."""
+    B, M, Hq, K = q.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    ts = (q, k_new, v_new, k_cache, v_cache)
+    if q.dtype not in _DTYPE or any(t.dtype != q.dtype for t in ts):
+        raise ValueError("q, k_new, v_new, k_cache, v_cache must share dtype float16 or bfloat16")
+    if tuple(k_new.shape) != (B, M, Hkv, K) or tuple(v_new.shape) != (B, M, Hkv, K):
+        raise ValueError("k_new and v_new must be [B, M, Hkv, K]")
+    if tuple(k_cache.shape) != (B, cap, Hkv, K) or tuple(v_cache.shape) != (B, cap, Hkv, K):
+        raise ValueError("k_cache and v_cache must be [B, cap, Hkv, K]")
+    for name, t in (("cache_seqlens", cache_seqlens), ("q_seqlens", q_seqlens)):
+        if t is not None and (t.dtype != torch.int32 or not t.is_cuda or t.numel() != B):
+            raise ValueError(f"{name} must be an int32 CUDA tensor of B entries")
+    scale = K ** -0.5 if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, M, Hq, K), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, M), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [B, Hq, M] tensor")
+    rc = lib.mea_prefill_chunk(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(cache_seqlens), _ptr(q_seqlens), _ptr(out), _ptr(lse), B, M,
+                               cap, Hq, Hkv, K, _bmhk_strides(q, "q"),
+                               _bmhk_strides(k_new, "k_new"), _bmhk_strides(v_new, "v_new"),
+                               _bmhk_strides(k_cache, "k_cache"),
+                               _bmhk_strides(v_cache, "v_cache"), _bmhk_strides(out, "out"),
+                               _DTYPE[q.dtype], int(bool(causal)), int(bool(alibi)), scale,
+                               _stream(stream))
+    _check("mea_prefill_chunk", rc)
     return out, lse
 
 

@@ -201,6 +201,79 @@ int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
 
 int mea_sparse_block_size(void) { return mea::kSparseBlock; }
 
+int mea_prefill_chunk(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                      void* v_cache, const int32_t* cache_seqlens, const int32_t* q_seqlens,
+                      void* out, float* lse, int B, int M, int cache_rows, int Hq, int Hkv,
+                      int K, const int64_t q_strides[3], const int64_t kn_strides[3],
+                      const int64_t vn_strides[3], const int64_t kc_strides[3],
+                      const int64_t vc_strides[3], const int64_t o_strides[3],
+                      mea_dtype_t dtype, int causal, int alibi, float scale,
+                      cudaStream_t stream) {
+  if (B < 0 || M < 0 || cache_rows < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    return MEA_ERR_INVALID_ARG;
+  if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return MEA_ERR_INVALID_ARG;
+  if (!q_strides || !kn_strides || !vn_strides || !kc_strides || !vc_strides || !o_strides)
+    return MEA_ERR_INVALID_ARG;
+  if (!(scale == scale)) return MEA_ERR_INVALID_ARG;
+  if (B == 0 || M == 0) return MEA_OK;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_seqlens || !out)
+    return MEA_ERR_INVALID_ARG;
+  if (cache_rows < 1) return MEA_ERR_INVALID_ARG;
+  if (K != 64 && K != 128) return MEA_ERR_UNSUPPORTED;
+  if (scale < 0.f) return MEA_ERR_UNSUPPORTED;
+  for (const void* p : {q, k_new, v_new, static_cast<const void*>(k_cache),
+                        static_cast<const void*>(v_cache), static_cast<const void*>(out)})
+    if (!aligned16(p)) return MEA_ERR_UNSUPPORTED;
+  for (const int64_t* st : {q_strides, kn_strides, vn_strides, kc_strides, vc_strides, o_strides})
+    if (!strides_ok(st)) return MEA_ERR_UNSUPPORTED;
+  int* status = status_word();
+  if (!status) return MEA_ERR_CUDA;
+
+  mea::FwdLaunch L{};
+  const bool bf16 = dtype == MEA_BF16;
+  if (!encode_bmhk(&L.tmQ, q, bf16, B, M, Hq, K, q_strides, 128) ||
+      !encode_bmhk(&L.tmK, k_cache, bf16, B, cache_rows, Hkv, K, kc_strides, 128) ||
+      !encode_bmhk(&L.tmV, v_cache, bf16, B, cache_rows, Hkv, K, vc_strides, 128) ||
+      !encode_bmhk(&L.tmKn, k_new, bf16, B, M, Hkv, K, kn_strides, 128) ||
+      !encode_bmhk(&L.tmVn, v_new, bf16, B, M, Hkv, K, vn_strides, 128))
+    return MEA_ERR_CUDA;
+  mea::FwdArgs& a = L.args;
+  a.out = out;
+  a.lse = lse;
+  a.status = status;
+  a.o_sb = o_strides[0];
+  a.o_sm = o_strides[1];
+  a.o_sh = o_strides[2];
+  a.B = B;
+  a.M = M;
+  a.N = cache_rows;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.group = Hq / Hkv;
+  a.num_units = B;
+  a.num_mblocks = (M + mea::kFwdRowsPerCta - 1) / mea::kFwdRowsPerCta;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.cache_len = cache_seqlens;
+  a.q_lens = q_seqlens;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  for (int i = 0; i < 3; ++i) {
+    a.kn_s[i] = kn_strides[i];
+    a.vn_s[i] = vn_strides[i];
+    a.kc_s[i] = kc_strides[i];
+    a.vc_s[i] = vc_strides[i];
+  }
+  a.cap = cache_rows;
+  L.head_dim = K;
+  L.bf16 = bf16;
+  L.mask = causal ? static_cast<int>(MEA_BIAS_CAUSAL) : static_cast<int>(MEA_BIAS_NONE);
+  L.alibi = alibi != 0;
+  return mea::launch_fwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
 int mea_fwd_block_sparse(const void* q, const void* k, const void* v, void* out, float* lse,
                          int B, int M, int N, int Hq, int Hkv, int K,
                          const int64_t q_strides[3], const int64_t k_strides[3],

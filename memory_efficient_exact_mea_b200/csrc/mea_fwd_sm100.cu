@@ -35,6 +35,7 @@
 namespace mea {
 namespace {
 
+constexpr int kModeDense = 0, kModeSparse = 1, kModeCache = 2;
 constexpr int kBM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;        // keys per tile
 constexpr int kThreads = 608;
@@ -85,13 +86,27 @@ __device__ long long g_trace[kTraceCtas * kTraceSlots];
   } while (0)
 #endif
 
-// SPARSE: a block mask (one byte per 128-query x 128-key block) leaves out
-// whole score tiles ("FlashAttention (2022)", "Cosa mostravano i numeri": the
-// block-sparse variant); a left-out tile is neither loaded nor multiplied.
-template <int D, bool BF16, int MASK, bool ALIBI, bool SPARSE>
+// MODE kModeSparse: a block mask (one byte per 128-query x 128-key block)
+// leaves out whole score tiles ("FlashAttention (2022)", "Cosa mostravano i
+// numeri": the block-sparse variant); a left-out tile is neither loaded nor
+// multiplied.
+// MODE kModeCache: one prefill chunk against a KV cache ("Transformer :
+// comprendre l'entrainement et l'inference", "Pre-remplissage et decodage" and
+// "Un cache KV simple"): the chunk's queries attend to the cached rows
+// [0, past) (tmK/tmV over the cache) and to the chunk's own new rows (tmKn/tmVn
+// over the new keys/values) at positions past + r, and the CTAs copy the new
+// rows into the cache at [past, past + n).  Nothing in the launch reads a cache
+// row at or after past, so the copy races with no load.  The last tile of each
+// region is shifted back to end at the region's end (its first columns, seen by
+// an earlier tile or before row 0, are masked), so no row beyond a sequence's
+// valid rows is ever loaded.
+template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKn,
+               const __grid_constant__ CUtensorMap tmVn, const FwdArgs a) {
+  constexpr bool SPARSE = (MODE == kModeSparse);
+  constexpr bool kCache = (MODE == kModeCache);
   using L = Smem<D>;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
@@ -153,11 +168,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       return;
     }
   }
+  int past = 0;  // cache mode: rows cached before this chunk
+  if constexpr (kCache) {
+    past = a.cache_len[unit];
+    q_len = a.q_lens ? a.q_lens[unit] : a.M;
+    if (past < 0 || q_len < 0 || q_len > a.M || past > a.cap - q_len) {
+      if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
+      return;
+    }
+    k_len = past + q_len;
+    // The append: the CTAs of one (sequence, kv head) -- its query heads times
+    // its query blocks -- each copy an equal share of the new rows.
+    const int slices = a.group * a.num_mblocks;
+    const int slice = (h % a.group) * a.num_mblocks + static_cast<int>(blockIdx.x % a.num_mblocks);
+    const long long r0 = static_cast<long long>(q_len) * slice / slices;
+    const long long r1 = static_cast<long long>(q_len) * (slice + 1) / slices;
+    constexpr int kPieces = D / 8;  // 16-byte pieces per row
+    for (long long e = threadIdx.x; e < (r1 - r0) * kPieces * 2; e += kThreads) {
+      const int kv = static_cast<int>(e & 1);
+      const long long r = r0 + (e >> 1) / kPieces;
+      const int c = static_cast<int>((e >> 1) % kPieces);
+      const long long* ns = kv ? a.vn_s : a.kn_s;
+      const long long* cs = kv ? a.vc_s : a.kc_s;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          static_cast<const uint16_t*>(kv ? a.v_new : a.k_new) + unit * ns[0] + r * ns[1] +
+          kvh * ns[2] + c * 8);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(kv ? a.v_cache : a.k_cache) +
+                                            unit * cs[0] + (past + r) * cs[1] + kvh * cs[2] +
+                                            c * 8);
+      *dst = *src;
+    }
+  }
   const int m_base = mb * kFwdRowsPerCta;
   if (m_base >= q_len) return;
   const int off = k_len - q_len;  // bottom-right causal alignment
 
-  // Key tiles each query tile needs.
+  // Key tiles each query tile needs.  Cache mode: the past tiles (all visible)
+  // then the new tiles (up to the diagonal under a causal mask).
+  const int n_past_tiles = kCache ? (past + kBN - 1) / kBN : 0;
+  const int n_new_tiles = kCache ? (q_len + kBN - 1) / kBN : 0;
   int nt_tile[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
@@ -168,8 +217,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kCausal) nkeys = min(k_len, max(0, mt + kBM + off));
     }
     nt_tile[t] = (nkeys + kBN - 1) / kBN;
+    if constexpr (kCache) {
+      const int nn = mt < q_len ? (kCausal ? min(q_len, mt + kBM) : q_len) : 0;
+      nt_tile[t] = mt < q_len ? n_past_tiles + (nn + kBN - 1) / kBN : 0;
+    }
   }
   const int nt = max(nt_tile[0], nt_tile[1]);
+
+  // Key tile j: the row its copy starts at (in the cache or in the new rows),
+  // the key position of its column 0 and its first column not already seen by
+  // an earlier tile (or not before row 0).  Only the last tile of a region is
+  // shifted back.
+  struct KeyTile {
+    int row, pos, lo;
+    bool fresh;
+  };
+  auto key_tile = [&](int j) -> KeyTile {
+    if constexpr (kCache) {
+      if (j < n_past_tiles) {
+        const bool last = j == n_past_tiles - 1;
+        const int r = last ? past - kBN : j * kBN;
+        return {r, r, last ? n_past_tiles * kBN - past : 0, false};
+      }
+      const int m = j - n_past_tiles;
+      const bool last = m == n_new_tiles - 1;
+      const int r = last ? q_len - kBN : m * kBN;
+      return {r, past + r, last ? n_new_tiles * kBN - q_len : 0, true};
+    }
+    return {k0 + j * kBN, j * kBN, 0, false};
+  };
 
   // Does query tile t compute key tile j?  Every role walks the key tiles in
   // the same order and skips those neither query tile needs; the barriers of a
@@ -213,6 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if constexpr (kCache) {
+      tma_prefetch_desc(&tmKn);
+      tma_prefetch_desc(&tmVn);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -232,14 +312,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (SPARSE) {
           if (!uses(0, j) && !uses(1, j)) continue;
         }
+        const KeyTile kt = key_tile(j);
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = it % S;
           if (!mbar_wait(&kv_empty[slot], ((it / S) & 1) ^ 1, abort_flag, a.status)) break;
           mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
           const CUtensorMap* map = kv ? &tmV : &tmK;
+          if (kCache && kt.fresh) map = kv ? &tmVn : &tmKn;
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
-                        c * 64, kvh, k0 + j * kBN, bidx);
+                        c * 64, kvh, kt.row, bidx);
         }
         if (*abort_flag) break;
       }
@@ -473,10 +555,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // Keys this row may see in the tile: columns [0, limit).  Tiles that need
       // no masking for any row of the warp take the unmasked path (warp-uniform).
-      const int n0 = j * kBN;
+      // Cache mode: columns before kfirst were seen by an earlier tile.
+      int n0 = j * kBN, kfirst = 0;
+      if constexpr (kCache) {
+        const KeyTile kt = key_tile(j);
+        n0 = kt.pos;
+        kfirst = kt.lo;
+      }
       int limit = k_len - n0;
       if (kCausal) limit = min(limit, pos_i + 1 - n0);
-      const bool masked = __any_sync(0xffffffffu, limit < kBN);
+      const bool masked = __any_sync(0xffffffffu, limit < kBN) || (kCache && kfirst > 0);
+      // Column i of this thread is outside [kfirst, limit).
+      auto hidden = [&](int i) -> bool {
+        if constexpr (kCache) return c0 + i >= limit || c0 + i < kfirst;
+        return c0 + i >= limit;
+      };
       const float dpos0 = static_cast<float>(n0 + c0 - pos_i);  // ALiBi distance of column c0
       tmem_ld_wait(sr[0]);
       tmem_ld_wait(sr[1]);
@@ -494,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBN / 2; ++i) {
           float y = fmaf(__uint_as_float(sr[i >> 5][i & 31]), a.scale_log2,
                          -slope_log2 * fabsf(dpos0 + static_cast<float>(i)));
-          if (masked && c0 + i >= limit) y = neg_inf();
+          if (masked && hidden(i)) y = neg_inf();
           sr[i >> 5][i & 31] = __float_as_uint(y);
           mx[i & 3] = fmaxf(mx[i & 3], y);
         }
@@ -506,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
 #pragma unroll
         for (int i = 0; i < kBN / 2; ++i)
-          if (c0 + i < limit) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i >> 5][i & 31]));
+          if (!hidden(i)) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i >> 5][i & 31]));
       }
       float pmax = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       if constexpr (!ALIBI) pmax = (pmax == neg_inf()) ? pmax : pmax * a.scale_log2;
@@ -534,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const f2 y = ALIBI ? add2(v, nsub2) : fma2(v, scale2, nsub2);
         f2 p = {ex2(y.x), ex2(y.y)};
         if (!ALIBI && masked) {
-          if (c0 + i >= limit) p.x = 0.f;
-          if (c0 + i + 1 >= limit) p.y = 0.f;
+          if (hidden(i)) p.x = 0.f;
+          if (hidden(i + 1)) p.y = 0.f;
         }
         ps[(i >> 1) & 1] = add2(ps[(i >> 1) & 1], p);
         sr[i >> 5][i & 31] = __float_as_uint(p.x);
@@ -647,9 +740,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool BF16, int MASK, bool ALIBI, bool SPARSE = false>
+template <int D, bool BF16, int MASK, bool ALIBI, int MODE = kModeDense>
 cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
-  auto kern = fwd_kernel<D, BF16, MASK, ALIBI, SPARSE>;
+  auto kern = fwd_kernel<D, BF16, MASK, ALIBI, MODE>;
   const int smem = Smem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -657,7 +750,8 @@ cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
                          L.args.num_units;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.args);
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmKn,
+                                                                  L.tmVn, L.args);
   return cudaGetLastError();
 }
 
@@ -665,10 +759,19 @@ template <int D, bool BF16>
 cudaError_t dispatch_mask(const FwdLaunch& L, cudaStream_t s) {
   if (L.args.block_mask != nullptr) {  // block-sparse: no mask or causal only
     switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
-      case 0: return launch_t<D, BF16, 0, false, true>(L, s);
-      case 1: return launch_t<D, BF16, 0, true, true>(L, s);
-      case 2: return launch_t<D, BF16, 1, false, true>(L, s);
-      case 3: return launch_t<D, BF16, 1, true, true>(L, s);
+      case 0: return launch_t<D, BF16, 0, false, kModeSparse>(L, s);
+      case 1: return launch_t<D, BF16, 0, true, kModeSparse>(L, s);
+      case 2: return launch_t<D, BF16, 1, false, kModeSparse>(L, s);
+      case 3: return launch_t<D, BF16, 1, true, kModeSparse>(L, s);
+    }
+    return cudaErrorInvalidValue;
+  }
+  if (L.args.cache_len != nullptr) {  // prefill chunk against a cache: no mask or causal
+    switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
+      case 0: return launch_t<D, BF16, 0, false, kModeCache>(L, s);
+      case 1: return launch_t<D, BF16, 0, true, kModeCache>(L, s);
+      case 2: return launch_t<D, BF16, 1, false, kModeCache>(L, s);
+      case 3: return launch_t<D, BF16, 1, true, kModeCache>(L, s);
     }
     return cudaErrorInvalidValue;
   }

@@ -27,12 +27,24 @@ struct FwdArgs {
   const uint8_t* block_mask;
   long long bm_sb, bm_sh;
   int bm_nk;        // ceil(N / 128)
+  // Prefill chunk against a cache only (cache_len nullptr otherwise): the
+  // chunk's q/out/lse have M rows per sequence, of which q_lens[b] (nullptr: M)
+  // are real; the caches [B, cap, Hkv, K] hold cache_len[b] rows before the call.
+  const int32_t* cache_len;
+  const int32_t* q_lens;
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+  long long kn_s[3], vn_s[3], kc_s[3], vc_s[3];  // element strides (b, row, head)
+  int cap;
 };
 
 constexpr int kSparseBlock = 128;  // rows and keys per block-mask entry
 
 struct FwdLaunch {
   CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmKn, tmVn;  // new keys / values of a prefill chunk (cache mode only)
   FwdArgs args;
   int head_dim;   // 64 or 128
   bool bf16;

@@ -206,3 +206,59 @@ def block_sparse_noncausal(M: int = 4096) -> tuple[Prefill, torch.Tensor]:
     p = make_prefill(f"block_sparse_b8_h16_k64_f16_m{M}_d50", 8, M, M, 16, 16, 64, "f16", "none",
                      seed=1006)
     return p, block_mask(8, 16, M, M, 128, 0.5, seed=1007, keep_diagonal=True)
+
+
+@dataclass
+class Chunk:
+    """One prefill chunk against a KV cache: q [B,M,Hq,K], new k/v [B,M,Hkv,K],
+    caches [B,cap,Hkv,K] holding past[b] rows, q_lens[b] real rows per chunk."""
+
+    name: str
+    B: int
+    M: int
+    cap: int
+    Hq: int
+    Hkv: int
+    K: int
+    dtype: str
+    causal: bool
+    past: list
+    q_lens: list
+    alibi: bool = False
+    seed: int = 0
+    q: torch.Tensor = field(default=None, repr=False)
+    k_new: torch.Tensor = field(default=None, repr=False)
+    v_new: torch.Tensor = field(default=None, repr=False)
+    k_cache: torch.Tensor = field(default=None, repr=False)
+    v_cache: torch.Tensor = field(default=None, repr=False)
+
+    @property
+    def scale(self) -> float:
+        return self.K ** -0.5
+
+
+def make_chunk(name, past, M, cap, Hq, Hkv, K, dtype, causal, seed, q_lens=None,
+               alibi=False) -> Chunk:
+    """Cache rows [0, past[b]) and the chunk are N(0,1); cache rows from past[b] on
+    are filled with a constant 3.0 (they are overwritten or never read)."""
+    B = len(past)
+    q_lens = list(q_lens) if q_lens is not None else [M] * B
+    c = Chunk(name, B, M, cap, Hq, Hkv, K, dtype, causal, list(past), q_lens, alibi, seed)
+    g = generator(seed)
+    c.q = randn((B, M, Hq, K), dtype, g)
+    c.k_new = randn((B, M, Hkv, K), dtype, g)
+    c.v_new = randn((B, M, Hkv, K), dtype, g)
+    c.k_cache = torch.full((B, cap, Hkv, K), 3.0, dtype=DTYPES[dtype])
+    c.v_cache = torch.full((B, cap, Hkv, K), 3.0, dtype=DTYPES[dtype])
+    for b, p in enumerate(past):
+        c.k_cache[b, :p] = randn((p, Hkv, K), dtype, g)
+        c.v_cache[b, :p] = randn((p, Hkv, K), dtype, g)
+    return c
+
+
+def chunk_prefill() -> Chunk:
+    """Chunked prefill: B=8 sequences with U[1024, 8192] cached rows each take a
+    512-row chunk; Hq=32, Hkv=8, K=128, bf16, causal; cache capacity 8704 rows."""
+    past = lengths(8, 1024, 8192, generator(1008)).tolist()
+    return make_chunk("chunk512_b8_past1k-8k_hq32_hkv8_k128_bf16", past, 512, 8704, 32, 8, 128,
+                      "bf16", True, seed=1009)

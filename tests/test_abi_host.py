@@ -199,3 +199,27 @@ def test_block_sparse_rejects_bad_arguments(lib):
     assert call(ms=(-1, 0)) == INVALID
     assert call(ms=None) == INVALID
     assert call(K=96) == UNSUPPORTED
+
+
+def test_prefill_chunk_rejects_bad_arguments(lib):
+    INVALID, UNSUPPORTED = -1, -2
+    vp = ctypes.c_void_p
+
+    def call(B=2, M=64, cap=128, Hq=4, Hkv=2, K=64, dtype=0, causal=1, scale=0.1, cl=16, kc=16,
+             q=16):
+        s = I64x3(1 << 20, 1024, 128)
+        return lib.mea_prefill_chunk(vp(q), vp(16), vp(16), vp(kc), vp(16), vp(cl), None, vp(16),
+                                     None, B, M, cap, Hq, Hkv, K, s, s, s, s, s, s, dtype, causal,
+                                     0, ctypes.c_float(scale), None)
+    assert call(Hq=3) == INVALID
+    assert call(dtype=4) == INVALID
+    assert call(causal=2) == INVALID
+    assert call(cl=None) == INVALID
+    assert call(kc=None) == INVALID
+    assert call(cap=0) == INVALID
+    assert call(scale=float("nan")) == INVALID
+    assert call(K=80) == UNSUPPORTED
+    assert call(scale=-1.0) == UNSUPPORTED
+    assert call(q=8) == UNSUPPORTED
+    assert call(B=0) == 0
+    assert call(M=0) == 0
