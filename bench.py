@@ -107,25 +107,30 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources a kernel's compiled code depends on (for matching a recorded ncu
+# capture to the current build).
+KERNEL_SOURCES = {"fwd_sweep": ["mea_fwd_sm100.cu", "mea_internal.h", "sm100.cuh"]}
+
+
+def kernel_source_hash(kernel: str = "fwd_sweep") -> str:
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
+    for name in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel: str, scale_units: float | None = None):
+def traffic_for(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources."""
+    the kernel's current sources."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         t = json.load(f)
-    if t.get("source_hash") != kernel_source_hash():
-        return None
     e = t.get("kernels", {}).get(kernel)
-    return None if e is None else e.get("bytes_per_launch")
+    if e is None or e.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return e.get("bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------

@@ -435,6 +435,17 @@ extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* 
   if (!status) return MEA_ERR_CUDA;
 
   mea::BwdLaunch L{};
+  const bool bf16 = dtype == MEA_BF16;
+  if (M > 0 && N > 0) {
+    const int64_t sq[3] = {static_cast<int64_t>(M) * Hq * K, static_cast<int64_t>(Hq) * K, K};
+    const int64_t sk[3] = {static_cast<int64_t>(N) * Hkv * K, static_cast<int64_t>(Hkv) * K, K};
+    const int bm = mea::bwd_query_block(K);
+    if (!encode_bmhk(&L.tmQ, q, bf16, B, M, Hq, K, sq, bm) ||
+        !encode_bmhk(&L.tmDO, dout, bf16, B, M, Hq, K, sq, bm) ||
+        !encode_bmhk(&L.tmK, k, bf16, B, N, Hkv, K, sk, mea::kBwdBlock) ||
+        !encode_bmhk(&L.tmV, v, bf16, B, N, Hkv, K, sk, mea::kBwdBlock))
+      return MEA_ERR_CUDA;
+  }
   mea::BwdArgs& a = L.args;
   a.q = q;
   a.k = k;
@@ -464,19 +475,15 @@ extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* 
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   L.head_dim = K;
-  L.bf16 = dtype == MEA_BF16;
+  L.bf16 = bf16;
   L.mask = static_cast<int>(bias);
   L.alibi = alibi != 0;
-  if (N > 0 && M == 0) {  // no query rows: dk = dv = 0
-    if (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess ||
-        cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess)
-      return MEA_ERR_CUDA;
-    return MEA_OK;
-  }
-  if (N > 0 && (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) !=
-                    cudaSuccess ||
-                cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) !=
-                    cudaSuccess))
+  // The kernel writes every key row of every sequence; rows no sequence owns
+  // (packed batches) and the no-query case are zeroed here.
+  if (N > 0 && (M == 0 || packed) &&
+      (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess ||
+       cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess))
     return MEA_ERR_CUDA;
+  if (M == 0) return MEA_OK;
   return mea::launch_bwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
 }

@@ -84,7 +84,7 @@ struct DecodeLaunch {
 cudaError_t launch_decode(const DecodeLaunch& launch, cudaStream_t stream);
 
 // Backward: dq, dk, dv from q, k, v, out, dout and the forward's lse.
-constexpr int kBwdBlock = 64;  // query rows and key rows per tile
+constexpr int kBwdBlock = 128;  // keys per CTA
 
 struct BwdArgs {
   const void *q, *k, *v, *out, *dout;  // contiguous [B,M,Hq,K] / [B,N,Hkv,K]
@@ -100,6 +100,7 @@ struct BwdArgs {
 };
 
 struct BwdLaunch {
+  CUtensorMap tmQ, tmK, tmV, tmDO;  // boxes: bwd_query_block rows (q, dout), kBwdBlock rows (k, v)
   BwdArgs args;
   int head_dim;
   bool bf16;
@@ -108,5 +109,8 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_bwd(const BwdLaunch& launch, cudaStream_t stream);
+
+// Query rows per step of the backward kernel for head dimension 64 or 128.
+int bwd_query_block(int head_dim);
 
 }  // namespace mea

@@ -215,6 +215,30 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int m, int n, bool b
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// The same with A stored M-contiguous too (a_mn_major, bit 15): both operands
+// may then be "transposed" views of row-major shared tiles.
+__host__ __device__ constexpr uint32_t idesc_f16_ab(bool bf16, int m, int n, bool a_mn_major,
+                                                    bool b_mn_major) {
+  return idesc_f16(bf16, m, n, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Makes this thread's ordinary shared-memory stores visible to the async proxy
+// (tcgen05.mma operand reads, TMA) for whoever synchronises with it afterwards.
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Fire-and-forget fp32 additions to global memory.
+__device__ __forceinline__ void red_add(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread t of the warp gets lane
 // (warp's lane quarter) + t, columns [col, col + 32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
