@@ -60,6 +60,25 @@ bool encode_bmhk(CUtensorMap* map, const void* base, bool bf16, int batch, int r
   return r == CUDA_SUCCESS;
 }
 
+// A contiguous fp32 [batch, rows, heads, K] tensor as a rank-4 TMA map with
+// 32-element x 1 head x `box_rows` boxes and 128-byte swizzle (reduction target).
+bool encode_f32_bmhk(CUtensorMap* map, void* base, int batch, int rows, int heads, int K,
+                     int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(K) * 4,
+                                 static_cast<cuuint64_t>(heads) * K * 4,
+                                 static_cast<cuuint64_t>(rows) * heads * K * 4};
+  const cuuint32_t box[4] = {32, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A packed cache [rows, heads, K] (contiguous) as a rank-3 TMA map.
 bool encode_cache(CUtensorMap* map, const void* base, bool bf16, int rows, int heads, int K,
                   int box_rows) {
@@ -443,7 +462,8 @@ extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* 
     if (!encode_bmhk(&L.tmQ, q, bf16, B, M, Hq, K, sq, bm) ||
         !encode_bmhk(&L.tmDO, dout, bf16, B, M, Hq, K, sq, bm) ||
         !encode_bmhk(&L.tmK, k, bf16, B, N, Hkv, K, sk, mea::kBwdBlock) ||
-        !encode_bmhk(&L.tmV, v, bf16, B, N, Hkv, K, sk, mea::kBwdBlock))
+        !encode_bmhk(&L.tmV, v, bf16, B, N, Hkv, K, sk, mea::kBwdBlock) ||
+        !encode_f32_bmhk(&L.tmDQ, workspace, B, M, Hq, K, bm))
       return MEA_ERR_CUDA;
   }
   mea::BwdArgs& a = L.args;

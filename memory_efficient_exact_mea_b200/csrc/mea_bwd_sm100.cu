@@ -19,16 +19,25 @@
 // bwd_kernel, per query block i of BM rows (BM = 64 at K = 128, 128 at K = 64),
 // with the block's keys on the 128 TMEM lanes:
 //   S^T  = K Q_i^T,  dP^T = V dO_i^T                  (tcgen05, both operands K-major)
-//   P^T, dS^T from S^T, dP^T, lse_i, D_i               (128 threads, one per key)
-//     P^T (16-bit) is written back over S^T in TMEM, dS^T to shared memory
+//   P^T, dS^T from S^T, dP^T, lse_i, D_i               (256 threads, two per key)
+//     P^T (16-bit) to its own TMEM columns, dS^T to shared memory (two buffers)
 //   dV  += P^T dO_i   (A = P^T from TMEM)              dK += dS^T Q_i
 //   dQ_i = dS_i K  (K = 64)  or  dQ_i^T = K^T dS_i^T (K = 128): both M = 128, N = 64
-//   dQ_i is drained by four warps into the fp32 accumulator with global reductions.
-// TMEM columns: S^T [0, BM) | dP^T [BM, 2BM) | dQ [2BM, 2BM+64) | dV (K) | dK (K).
+//   dQ_i is drained by four warps: scaled, staged in shared memory -- in the
+//   Q_i/dO_i stage, which no MMA reads any more -- and added to the fp32
+//   accumulator by TMA tensor reductions (one per 32 columns); the stage is
+//   handed back to the loader once the reductions have read it.
+// The S^T / dP^T columns are released as soon as the P/dS threads have read
+// them, so the MMA thread issues the next block's S^T, dP^T before this block's
+// dV, dK, dQ and the P/dS arithmetic of one block overlaps the MMAs of its
+// neighbours.  dS^T of block i goes to buffer i % 2, last read by block i-2's
+// MMAs, which completed before block i's S^T did (issue order); P^T of block i
+// is stored once block i-1's MMAs are done.
 //
-// CTA (320 threads): warps 0-3 P/dS and the dK/dV epilogue, warps 4-7 the dQ
-// drain, warp 8 allocates TMEM and one of its threads issues every MMA, warp 9
-// loads (one thread issues the TMA copies; the warp stages lse and D of each block).
+// CTA (448 threads): warps 0-7 P/dS and the dK/dV epilogue (warps w and w+4
+// share TMEM lane quarter w, each taking half of the query columns), warps 8-11
+// the dQ drain, warp 12 allocates TMEM and one of its threads issues every MMA,
+// warp 13 loads (one thread issues the TMA copies; the warp stages lse and D).
 #include <math.h>
 
 #include <algorithm>
@@ -40,14 +49,42 @@ namespace mea {
 namespace {
 
 constexpr int kBN = kBwdBlock;  // keys per CTA (= TMEM lanes)
-constexpr int kThreads = 320;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kThreads = 448;
+constexpr int kDrainWarp = 8;  // warps 8..11
+constexpr int kMmaWarp = 12;
+constexpr int kLoadWarp = 13;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
-__device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
+
+// Pipeline timeline for performance work: built only with -DMEA_TRACE, it
+// records clock64() at pipeline events of the first kBwdTraceCtas CTAs.
+// Slots per CTA: step s (< 64), event e (< 32) -> s*32 + e; CTA-level events at
+// 2048 + e.
+#ifdef MEA_TRACE
+constexpr int kBwdTraceCtas = 4;
+constexpr int kBwdTraceSlots = 2048 + 32;
+__device__ long long g_bwd_trace[kBwdTraceCtas * kBwdTraceSlots];
+#define BWD_TRACE(s, e)                                                                   \
+  do {                                                                                    \
+    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);      \
+    const int slot_ = (s) < 64 ? (s) * 32 + (e) : -1;                                     \
+    if (cta_ < kBwdTraceCtas && slot_ >= 0) g_bwd_trace[cta_ * kBwdTraceSlots + slot_] = clock64(); \
+  } while (0)
+#define BWD_TRACE_CTA(e)                                                                  \
+  do {                                                                                    \
+    const int cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);      \
+    if (cta_ < kBwdTraceCtas) g_bwd_trace[cta_ * kBwdTraceSlots + 2048 + (e)] = clock64(); \
+  } while (0)
+#else
+#define BWD_TRACE(s, e) \
+  do {                  \
+  } while (0)
+#define BWD_TRACE_CTA(e) \
+  do {                   \
+  } while (0)
+#endif
 
 template <bool BF16>
 __device__ __forceinline__ float to_f(uint16_t x) {
@@ -64,23 +101,31 @@ struct BwdCfg {
   static constexpr int kKVTile = kChunksD * kKVChunk;
   static constexpr int kQTile = kChunksD * kQChunk;
   static constexpr int kDSTile = (BM / 64) * kKVChunk;  // dS^T: 128 keys x BM queries
+  static constexpr int kStages = 3;                   // Q / dO stages
+  static constexpr int kStage = 2 * kQTile;           // Q then dO
+  static constexpr int kDQSBox = BM * 128;            // dQ staging: D/32 boxes of BM x 128 B
+  static_assert((D / 32) * kDQSBox == kStage, "dQ staging fills one Q/dO stage");
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kK = 0;
   static constexpr int kV = kKVTile;
-  static constexpr int kQ = 2 * kKVTile;              // two stages
-  static constexpr int kDO = kQ + 2 * kQTile;         // two stages
-  static constexpr int kDS = kDO + 2 * kQTile;
-  static constexpr int kLse = kDS + kDSTile;          // [2][BM] lse * log2(e) (+inf: no weight)
-  static constexpr int kDelta = kLse + 2 * BM * 4;    // [2][BM]
-  static constexpr int kBar = kDelta + 2 * BM * 4;
-  static constexpr int kNumBars = 10;
+  static constexpr int kQD = 2 * kKVTile;              // stage i: Q at kQD + i*kStage, dO after it
+  static constexpr int kDS = kQD + kStages * kStage;   // two buffers (step parity)
+  static constexpr int kLse = kDS + 2 * kDSTile;      // [stage][BM] -lse * log2(e) (-inf: no weight)
+  static constexpr int kDelta = kLse + kStages * BM * 4;  // [stage][BM] -D
+  static constexpr int kBar = kDelta + kStages * BM * 4;
+  static constexpr int kNumBars = 14;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;
-  // tensor memory columns
-  static constexpr uint32_t kColS = 0, kColDP = BM, kColDQ = 2 * BM, kColDV = 2 * BM + 64,
-                            kColDK = 2 * BM + 64 + D;
-  static_assert(kColDK + D <= kTmemCols, "tensor memory layout");
+  // tensor memory columns (every region starts on a multiple of 64):
+  //   K = 64:  S^T 0 | dP^T 128 | P^T 256 (64) | dQ 320 | dV 384 | dK 448
+  //   K = 128: S^T 0 | dP^T 64 | dQ 128 | dV 192 | dK 320 | P^T 448 (32)
+  static constexpr uint32_t kColS = 0, kColDP = BM;
+  static constexpr uint32_t kColP = (D == 64) ? 256 : 448;
+  static constexpr uint32_t kColDQ = (D == 64) ? 320 : 128;
+  static constexpr uint32_t kColDV = (D == 64) ? 384 : 192;
+  static constexpr uint32_t kColDK = (D == 64) ? 448 : 320;
+  static_assert(kColDK + D <= kTmemCols && kColP + BM / 2 <= kTmemCols, "tensor memory layout");
 };
 
 // One warp per (row, query head): D = <dout, out>, and zero the dq accumulator row.
@@ -119,7 +164,7 @@ template <int D, bool BF16, int MASK, bool ALIBI>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-               const BwdArgs a) {
+               const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
   using C = BwdCfg<D>;
   constexpr int BM = C::BM;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
@@ -129,14 +174,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  constexpr int NS = C::kStages;
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;    // [2] Q, dO (+ lse, D) of a step landed
-  uint64_t* q_empty = bars + 3;   // [2] every MMA reading the stage completed
-  uint64_t* s_full = bars + 5;    // S^T, dP^T of the step are in TMEM
-  uint64_t* p_ready = bars + 6;   // P^T in TMEM and dS^T in shared memory (128 arrivals)
-  uint64_t* dq_full = bars + 7;   // dQ of the step is in TMEM
-  uint64_t* dq_empty = bars + 8;  // dQ read out of TMEM (128 arrivals)
-  uint64_t* mma_done = bars + 9;
+  uint64_t* q_full = bars + 1;        // [NS] Q, dO (+ lse, D) of a step landed
+  uint64_t* q_empty = bars + 1 + NS;  // [NS] the stage is free again (its dQ reductions read it)
+  uint64_t* s_full = bars + 1 + 2 * NS;   // S^T, dP^T of the step are in TMEM
+  uint64_t* s_free = s_full + 1;      // S^T, dP^T read out of TMEM (256 arrivals)
+  uint64_t* p_ready = s_full + 2;     // P^T in TMEM and dS^T in shared memory (256 arrivals)
+  uint64_t* p_done = s_full + 3;      // the step's dV, dK, dQ MMAs completed
+  uint64_t* dq_full = s_full + 4;     // dQ of the step is in TMEM
+  uint64_t* dq_empty = s_full + 5;    // dQ read out of TMEM (128 arrivals)
+  uint64_t* mma_done = s_full + 6;
   float* s_lse = reinterpret_cast<float*>(smem + C::kLse);
   float* s_delta = reinterpret_cast<float*>(smem + C::kDelta);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemSlot);
@@ -170,12 +218,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_ready, 128);
+    mbar_init(s_free, 256);
+    mbar_init(p_ready, 256);
+    mbar_init(p_done, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(mma_done, 1);
@@ -196,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0) BWD_TRACE_CTA(0);
 
   if (warp == kLoadWarp) {
     // ===================== loads =============================================
@@ -211,39 +262,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < steps && ok; ++s) {
       const int h = kvh * a.group + s / n_mblocks;
       const int m0 = m_first + (s % n_mblocks) * BM;
-      const int slot = s & 1;
-      if (!(ok = mbar_wait_warp(&q_empty[slot], ((s >> 1) & 1) ^ 1, abort_flag, a.status))) break;
-      // lse (log2 units) and D of the block's rows; +inf marks a row that takes
-      // no weight (past the sequence, or no visible key in the forward).
-      for (int r = lane; r < BM; r += 32) {
-        const int i = m0 + r;
-        float l2 = pos_inf(), dl = 0.f;
+      const int slot = s % NS;
+      // -lse (log2 units) and -D of the block's rows, fetched before waiting for
+      // the stage; -inf marks a row that takes no weight (past the sequence, or
+      // no visible key in the forward).
+      float l2[BM / 32], dl[BM / 32];
+#pragma unroll
+      for (int u = 0; u < BM / 32; ++u) {
+        const int i = m0 + u * 32 + lane;
+        l2[u] = neg_inf();
+        dl[u] = 0.f;
         if (i < q_len) {
           const long long li = (static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + i;
-          const float l = a.lse[li];
-          if (l != neg_inf()) l2 = l * kLog2e;
-          dl = a.delta[li];
+          l2[u] = a.lse[li];
+          dl[u] = a.delta[li];
         }
-        s_lse[slot * BM + r] = l2;
-        s_delta[slot * BM + r] = dl;
+      }
+      if (!(ok = mbar_wait_warp(&q_empty[slot], ((s / NS) & 1) ^ 1, abort_flag, a.status))) break;
+      if (lane == 0) {
+        BWD_TRACE(s, 24);
+        mbar_expect_tx(&q_full[slot], C::kStage);
+        uint8_t* st = smem + C::kQD + slot * C::kStage;
+        for (int c = 0; c < C::kChunksD; ++c) {
+          tma_load_4d(st + c * C::kQChunk, &tmQ, &q_full[slot], c * 64, h, q0 + m0, bidx);
+          tma_load_4d(st + C::kQTile + c * C::kQChunk, &tmDO, &q_full[slot], c * 64, h, q0 + m0,
+                      bidx);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < BM / 32; ++u) {
+        s_lse[slot * BM + u * 32 + lane] = l2[u] == neg_inf() ? neg_inf() : -l2[u] * kLog2e;
+        s_delta[slot * BM + u * 32 + lane] = -dl[u];
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[slot], 2 * C::kQTile);
-        for (int c = 0; c < C::kChunksD; ++c) {
-          tma_load_4d(smem + C::kQ + slot * C::kQTile + c * C::kQChunk, &tmQ, &q_full[slot],
-                      c * 64, h, q0 + m0, bidx);
-          tma_load_4d(smem + C::kDO + slot * C::kQTile + c * C::kQChunk, &tmDO, &q_full[slot],
-                      c * 64, h, q0 + m0, bidx);
-        }
+        mbar_arrive(&q_full[slot]);
+        BWD_TRACE(s, 25);
       }
       issued = s + 1;
     }
     // Let every copy this warp started land before the CTA can exit.
     if (lane == 0 && steps > 0) {
       mbar_wait_drain(kv_full, 0, a.status);
-      for (int s = max(0, issued - 2); s < issued; ++s)
-        mbar_wait_drain(&q_full[s & 1], (s >> 1) & 1, a.status);
+      for (int s = max(0, issued - NS); s < issued; ++s)
+        mbar_wait_drain(&q_full[s % NS], (s / NS) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issue (one thread) ============================
@@ -252,19 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_g = idesc_f16_ab(BF16, kBN, D, false, true);
       constexpr uint32_t idesc_q = idesc_f16_ab(BF16, kBN, 64, true, true);
       const uint32_t sK = smem_u32(smem + C::kK), sV = smem_u32(smem + C::kV);
-      const uint32_t sDS = smem_u32(smem + C::kDS);
+      const uint32_t sDS0 = smem_u32(smem + C::kDS);
       const uint32_t tS = tmem_base + C::kColS, tDP = tmem_base + C::kColDP;
       const uint32_t tDQ = tmem_base + C::kColDQ, tDV = tmem_base + C::kColDV;
       const uint32_t tDK = tmem_base + C::kColDK;
-      bool ok = steps > 0 && mbar_wait(kv_full, 0, abort_flag, a.status);
-      for (int s = 0; s < steps && ok; ++s) {
-        const int slot = s & 1;
-        if (!(ok = mbar_wait(&q_full[slot], (s >> 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        const uint32_t sQ = smem_u32(smem + C::kQ + slot * C::kQTile);
-        const uint32_t sDO = smem_u32(smem + C::kDO + slot * C::kQTile);
-        // S^T = K Q^T and dP^T = V dO^T: K-major operands, 16 elements (32 bytes)
-        // per step inside a 128-byte swizzle row, then the next 64-column chunk.
+      const uint32_t tP = tmem_base + C::kColP;
+      // S^T = K Q^T and dP^T = V dO^T of step `st`: K-major operands, 16 elements
+      // (32 bytes) per step inside a 128-byte swizzle row, then the next chunk.
+      auto issue_s = [&](int st) {
+        const uint32_t sQ = smem_u32(smem + C::kQD + (st % NS) * C::kStage);
+        const uint32_t sDO = sQ + C::kQTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::kKVChunk + (kk & 3) * 32;
@@ -280,13 +339,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kk > 0);
         }
         umma_commit(s_full);
-        if (!(ok = mbar_wait(p_ready, s & 1, abort_flag, a.status))) break;
+      };
+      bool ok = steps > 0 && mbar_wait(kv_full, 0, abort_flag, a.status) &&
+                mbar_wait(&q_full[0], 0, abort_flag, a.status);
+      if (ok) {
+        BWD_TRACE_CTA(1);
         tc_fence_after();
+        issue_s(0);
+      }
+      for (int s = 0; s < steps && ok; ++s) {
+        const int slot = s % NS;
+        // The next block's scores go first: they only need its Q / dO and the
+        // S^T / dP^T columns, which the P/dS threads have read out.
+        if (s + 1 < steps) {
+          if (!(ok = mbar_wait(&q_full[(s + 1) % NS], ((s + 1) / NS) & 1, abort_flag, a.status)))
+            break;
+          BWD_TRACE(s, 0);
+          if (!(ok = mbar_wait(s_free, s & 1, abort_flag, a.status))) break;
+          BWD_TRACE(s, 1);
+          tc_fence_after();
+          issue_s(s + 1);
+          BWD_TRACE(s, 2);
+        }
+        if (!(ok = mbar_wait(p_ready, s & 1, abort_flag, a.status))) break;
+        BWD_TRACE(s, 3);
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(smem + C::kQD + slot * C::kStage);
+        const uint32_t sDO = sQ + C::kQTile;
+        const uint32_t sDS = sDS0 + (s & 1) * C::kDSTile;
         // dV += P^T dO (P^T from TMEM, two queries per column) and dK += dS^T Q:
         // dO and Q as N-contiguous B operands, 16 query rows (2048 bytes) per step.
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, C::kQChunk, 1024), idesc_g,
+          umma_ts(tDV, tP + kk * 8, sdesc_sw128(sDO + kk * 2048, C::kQChunk, 1024), idesc_g,
                   (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
@@ -295,10 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (s > 0 || kk > 0) ? 1u : 0u);
         // dQ: both operands M/N-contiguous views of row-major 128-key tiles, 16 keys
         // (2048 bytes) per step.  K = 128: dQ^T = K^T dS^T; K = 64: dQ = dS K.
+        BWD_TRACE(s, 4);
         if (s > 0) {
           if (!(ok = mbar_wait(dq_empty, (s - 1) & 1, abort_flag, a.status))) break;
           tc_fence_after();
         }
+        BWD_TRACE(s, 5);
         const uint32_t qa = (D == 128) ? sK : sDS;
         const uint32_t qb = (D == 128) ? sDS : sK;
 #pragma unroll
@@ -306,92 +393,132 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ss(tDQ, sdesc_sw128(qa + kk * 2048, C::kKVChunk, 1024),
                   sdesc_sw128(qb + kk * 2048, C::kKVChunk, 1024), idesc_q, kk > 0);
         umma_commit(dq_full);
-        umma_commit(&q_empty[slot]);
+        umma_commit(p_done);
+        BWD_TRACE(s, 6);
       }
       // Every MMA issued above has completed once this barrier flips.
       umma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, a.status);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ===================== P^T and dS^T, then the dK / dV epilogue ============
-    const int row = warp * 32 + lane;  // key inside the block = TMEM lane
+    constexpr int kCols = BM / 2;  // query columns per thread
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;  // key inside the block = TMEM lane
+    const int c0 = half * kCols;          // this thread's first query column
     const int j_loc = n0 + row;
     const bool key_ok = j_loc < k_len;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem_base + lane_addr + C::kColS;
-    const uint32_t tDP = tmem_base + lane_addr + C::kColDP;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem_base + lane_addr + C::kColS + c0;
+    const uint32_t tDP = tmem_base + lane_addr + C::kColDP + c0;
+    const uint32_t tP = tmem_base + lane_addr + C::kColP + c0 / 2;
     uint8_t* ds_row = smem + C::kDS + row * 128;
+    const f2 scale2 = {a.scale_log2, a.scale_log2};
+    const f2 zero2 = {0.f, 0.f};
     bool ok = true;
     for (int s = 0; s < steps && ok; ++s) {
       const int h = kvh * a.group + s / n_mblocks;
       const int m0 = m_first + (s % n_mblocks) * BM;
-      const int slot = s & 1;
+      const int slot = s % NS;
       float slope_log2 = 0.f;
       if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
-      // lse / D of this block were staged with the Q copy of the slot.
-      if (!(ok = mbar_wait_warp(&q_full[slot], (s >> 1) & 1, abort_flag, a.status))) break;
+      // -lse / -D of this block were staged with the Q copy of the stage.
+      if (!(ok = mbar_wait_warp(&q_full[slot], (s / NS) & 1, abort_flag, a.status))) break;
       if (!(ok = mbar_wait_warp(s_full, s & 1, abort_flag, a.status))) break;
+      const bool tracer = warp == 0 && lane == 0;
+      if (tracer) BWD_TRACE(s, 8);
       tc_fence_after();
-      const float* lse2 = s_lse + slot * BM;
-      const float* dlt = s_delta + slot * BM;
-#pragma unroll 1
-      for (int c = 0; c < BM / 32; ++c) {
-        uint32_t sr[32], dr[32];
+      // Per-element masks only where the tile reaches past the keys or past the
+      // diagonal for this thread's queries.
+      const bool full =
+          n0 + kBN <= k_len && (!kCausal || m0 + c0 + off >= n0 + kBN - 1);
+      const float* nl = s_lse + slot * BM + c0;
+      const float* nd = s_delta + slot * BM + c0;
+      uint8_t* ds_buf = ds_row + (s & 1) * C::kDSTile;
+      uint32_t pk[kCols / 2];
+      // 32 columns at a time: read S^T, dP^T out of TMEM (releasing them after the
+      // last chunk), then P = 2^(s*scale*log2e - lse*log2e) and dS = P (dP - D).
+#pragma unroll
+      for (int c = 0; c < kCols / 32; ++c) {
+        uint32_t sr[32], dr[32], dk[16];
         tmem_ld32(tS + 32 * c, sr);
         tmem_ld32(tDP + 32 * c, dr);
         tmem_ld_wait(sr);
         tmem_ld_wait(dr);
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float p2[2], d2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qc = 32 * c + k + e;    // query column
-            const int pos_i = m0 + qc + off;  // query position in key coordinates
-            float x = fmaf(__uint_as_float(sr[k + e]), a.scale_log2, -lse2[qc]);
-            if constexpr (ALIBI) x -= slope_log2 * fabsf(static_cast<float>(pos_i - j_loc));
-            bool vis = key_ok;
-            if constexpr (kCausal) vis = vis && j_loc <= pos_i;
-            const float p = vis ? ex2(x) : 0.f;
-            p2[e] = p;
-            d2[e] = p * (__uint_as_float(dr[k + e]) - dlt[qc]);
-          }
-          pk[k / 2] = pack2<BF16>(p2[0], p2[1]);
-          dk[k / 2] = pack2<BF16>(d2[0], d2[1]);
+        if (c == kCols / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(s_free);  // the next block's S^T / dP^T may be written now
+          if (tracer) BWD_TRACE(s, 9);
         }
-        // P^T over S^T columns already read: queries 2c', 2c'+1 in column c'.
-        tmem_st16(tS + 16 * c, pk);
-        // dS^T row `row`, columns 32c..32c+31, in the 128-byte-swizzled layout the
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int k = 32 * c + e;
+          const float2 l = *reinterpret_cast<const float2*>(nl + k);
+          const float2 dd = *reinterpret_cast<const float2*>(nd + k);
+          f2 x = fma2(f2{__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])}, scale2,
+                      f2{l.x, l.y});
+          const int pos = m0 + c0 + k + off;  // query position of column k, key coordinates
+          if constexpr (ALIBI) {
+            x.x -= slope_log2 * fabsf(static_cast<float>(pos - j_loc));
+            x.y -= slope_log2 * fabsf(static_cast<float>(pos + 1 - j_loc));
+          }
+          f2 p = {ex2(x.x), ex2(x.y)};
+          if (!full) {
+            bool v0 = key_ok, v1 = key_ok;
+            if constexpr (kCausal) {
+              v0 = v0 && j_loc <= pos;
+              v1 = v1 && j_loc <= pos + 1;
+            }
+            if (!v0) p.x = 0.f;
+            if (!v1) p.y = 0.f;
+          }
+          const f2 t = add2(f2{__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])},
+                            f2{dd.x, dd.y});
+          const f2 ds = fma2(p, t, zero2);
+          pk[k / 2] = pack2<BF16>(p.x, p.y);
+          dk[e / 2] = pack2<BF16>(ds.x, ds.y);
+        }
+        // dS^T row `row`, columns c0+32c .. +31, in the 128-byte-swizzled layout the
         // MMA descriptors read: 16-byte piece u of a 64-column chunk sits at u ^ (row & 7).
-        const int plane = (32 * c) >> 6;
+        const int col = c0 + 32 * c;
+        const int plane = col >> 6;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int piece = (((32 * c) & 63) >> 3) + u;
-          *reinterpret_cast<uint4*>(ds_row + plane * C::kKVChunk + ((piece ^ (row & 7)) << 4)) =
+          const int piece = ((col & 63) >> 3) + u;
+          *reinterpret_cast<uint4*>(ds_buf + plane * C::kKVChunk + ((piece ^ (row & 7)) << 4)) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
+      if (tracer) BWD_TRACE(s, 10);
+      // The previous block's dV MMAs still read P^T (queries 2c, 2c+1 in column c).
+      if (s > 0 && !(ok = mbar_wait_warp(p_done, (s - 1) & 1, abort_flag, a.status))) break;
+      if (tracer) BWD_TRACE(s, 11);
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kCols / 32; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(p_ready);
+      if (tracer) BWD_TRACE(s, 12);
     }
-    // ---- epilogue: dK (scaled) and dV of the valid keys ------------------------
+    // ---- epilogue: dK (scaled) and dV of the valid keys, half of K each -------
     // The TMEM loads are warp-collective: every lane issues them, and only the
     // global stores depend on the lane's key.
     if (ok) ok = mbar_wait_warp(mma_done, 0, abort_flag, a.status);
+    if (warp == 0 && lane == 0) BWD_TRACE_CTA(2);
     if (ok) {
       tc_fence_after();
+      const int dc0 = half * (D / 2);
       const long long grow = (static_cast<long long>(bidx) * a.N + k0 + j_loc) * a.Hkv + kvh;
-      uint8_t* dk_row = static_cast<uint8_t*>(a.dk) + grow * D * 2;
-      uint8_t* dv_row = static_cast<uint8_t*>(a.dv) + grow * D * 2;
+      uint8_t* dk_row = static_cast<uint8_t*>(a.dk) + (grow * D + dc0) * 2;
+      uint8_t* dv_row = static_cast<uint8_t*>(a.dv) + (grow * D + dc0) * 2;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t kr[32], vr[32];
         if (steps > 0) {
-          tmem_ld32(tmem_base + lane_addr + C::kColDK + 32 * c, kr);
-          tmem_ld32(tmem_base + lane_addr + C::kColDV + 32 * c, vr);
+          tmem_ld32(tmem_base + lane_addr + C::kColDK + dc0 + 32 * c, kr);
+          tmem_ld32(tmem_base + lane_addr + C::kColDV + dc0 + 32 * c, vr);
           tmem_ld_wait(kr);
           tmem_ld_wait(vr);
         } else {
@@ -417,52 +544,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ===================== dQ drain (warps 4-7) ===============================
+    // ===================== dQ drain (warps 8-11) ==============================
+    // dQ of a step goes TMEM -> registers (scaled) -> a 128-byte-swizzled staging
+    // tile in shared memory, whose 32-column boxes are added to the fp32
+    // accumulator by TMA reductions issued by one thread.
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // TMEM lane: a head dimension (K = 128) or a query (K = 64)
+    const bool leader = (warp == kDrainWarp && lane == 0);
     const uint32_t t_addr = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + C::kColDQ;
     bool ok = true;
     for (int s = 0; s < steps && ok; ++s) {
       const int h = kvh * a.group + s / n_mblocks;
       const int m0 = m_first + (s % n_mblocks) * BM;
       if (!(ok = mbar_wait_warp(dq_full, s & 1, abort_flag, a.status))) break;
+      if (leader) BWD_TRACE(s, 16);
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(t_addr, v0);
-      tmem_ld32(t_addr + 32, v1);
-      tmem_ld_wait(v0);
-      tmem_ld_wait(v1);
-      tc_fence_before();
-      mbar_arrive(dq_empty);
-      const long long row0 = (static_cast<long long>(bidx) * a.M + q0 + m0) * a.Hq + h;
-      if constexpr (D == 128) {
-        // lane = dimension `row`, columns = the block's 64 queries
-        const int nq = min(64, q_len - m0);
-        float* base = a.dq_acc + row0 * D + row;
-        const long long qstride = static_cast<long long>(a.Hq) * D;
+      // Stage dQ in this step's Q / dO stage: every MMA reading it has completed.
+      uint8_t* stage = smem + C::kQD + (s % NS) * C::kStage;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
+        uint32_t v[32];
+        tmem_ld32(t_addr + 32 * half, v);
+        tmem_ld_wait(v);
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+        }
+        if constexpr (D == 128) {
+          // lane = dimension `row`, columns = queries 32 half .. +31: element
+          // (query q, dim row) of box row/32 at row q, byte 4 (row % 32), swizzled.
+          uint8_t* box = stage + (row >> 5) * C::kDQSBox;
+          const int piece = (row & 31) >> 2, word = (row & 3) * 4;
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (k < nq) red_add(base + k * qstride, __uint_as_float(v0[k]) * a.scale);
+          for (int k = 0; k < 32; ++k) {
+            const int q = 32 * half + k;
+            const float x = (m0 + q < q_len) ? __uint_as_float(v[k]) * a.scale : 0.f;
+            *reinterpret_cast<float*>(box + q * 128 + ((piece ^ (k & 7)) << 4) + word) = x;
+          }
+        } else {
+          // lane = query m0 + row, columns = dims 32 half .. +31 = box `half`:
+          // 16-byte piece u at u ^ (row & 7).
+          const float sc = (m0 + row < q_len) ? a.scale : 0.f;
+          uint8_t* line = stage + half * C::kDQSBox + row * 128;
 #pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (32 + k < nq) red_add(base + (32 + k) * qstride, __uint_as_float(v1[k]) * a.scale);
-      } else {
-        // lane = query m0 + row, columns = its 64 dimensions
-        if (m0 + row < q_len) {
-          float* dst = a.dq_acc + (row0 + static_cast<long long>(row) * a.Hq) * D;
-#pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            red_add4(dst + k, __uint_as_float(v0[k]) * a.scale,
-                     __uint_as_float(v0[k + 1]) * a.scale, __uint_as_float(v0[k + 2]) * a.scale,
-                     __uint_as_float(v0[k + 3]) * a.scale);
-#pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            red_add4(dst + 32 + k, __uint_as_float(v1[k]) * a.scale,
-                     __uint_as_float(v1[k + 1]) * a.scale, __uint_as_float(v1[k + 2]) * a.scale,
-                     __uint_as_float(v1[k + 3]) * a.scale);
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<float4*>(line + ((u ^ (row & 7)) << 4)) =
+                make_float4(__uint_as_float(v[4 * u]) * sc, __uint_as_float(v[4 * u + 1]) * sc,
+                            __uint_as_float(v[4 * u + 2]) * sc, __uint_as_float(v[4 * u + 3]) * sc);
         }
       }
+      fence_async_smem();
+      named_sync(1, 128);
+      if (leader) {
+        BWD_TRACE(s, 17);
+#pragma unroll
+        for (int b = 0; b < D / 32; ++b)
+          tma_reduce_add_4d(&tmDQ, stage + b * C::kDQSBox, 32 * b, h, q0 + m0, bidx);
+        bulk_commit();
+        bulk_wait_read();
+        mbar_arrive(&q_empty[s % NS]);  // the loader may refill the stage
+      }
     }
+    if (leader) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -481,7 +624,7 @@ cudaError_t launch_main(const BwdLaunch& L, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const BwdArgs& a = L.args;
   dim3 grid(a.num_kblocks, a.Hkv, a.num_units);
-  kern<<<grid, kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmDO, a);
+  kern<<<grid, kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmDO, L.tmDQ, a);
   return cudaGetLastError();
 }
 
@@ -514,6 +657,14 @@ cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream) {
 }
 
 }  // namespace
+
+#ifdef MEA_TRACE
+// Copies the recorded backward timeline (kBwdTraceCtas x kBwdTraceSlots clock64 values).
+extern "C" int mea_bwd_trace_read(long long* host, int n) {
+  if (n > kBwdTraceCtas * kBwdTraceSlots) n = kBwdTraceCtas * kBwdTraceSlots;
+  return cudaMemcpyFromSymbol(host, g_bwd_trace, n * sizeof(long long)) == cudaSuccess ? n : -1;
+}
+#endif
 
 int bwd_query_block(int head_dim) { return head_dim == 128 ? BwdCfg<128>::BM : BwdCfg<64>::BM; }
 

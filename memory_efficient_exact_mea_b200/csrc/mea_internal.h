@@ -101,6 +101,7 @@ struct BwdArgs {
 
 struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // boxes: bwd_query_block rows (q, dout), kBwdBlock rows (k, v)
+  CUtensorMap tmDQ;                 // fp32 dq accumulator, 32 x 1 x bwd_query_block boxes
   BwdArgs args;
   int head_dim;
   bool bf16;
