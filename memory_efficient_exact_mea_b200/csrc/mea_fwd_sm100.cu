@@ -510,6 +510,201 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================== softmax warpgroups ===============================
+  if constexpr (kSepP) {
+    // Separate-P layout (K = 64, fp16): eight warps per query tile, each on 16
+    // TMEM lanes of its lane quarter (16x256b shape); a thread holds rows
+    // lane0 + t1 and lane0 + t1 + 8 and, of each 8-column group, the columns
+    // 2 t0 and 2 t0 + 1 (t0 = lane % 4, t1 = lane / 4).  The four threads of a
+    // row are lanes 4 t1 .. 4 t1 + 3 of one warp: row maxima and row sums
+    // combine with two shuffles.  P goes back as 16-bit pairs with the 16x128b
+    // shape, which puts keys 8k + 2 t0, 8k + 2 t0 + 1 into column 4k + t0.
+    const int t = warp >> 3;
+    const int wt = warp & 7, quarter = wt & 3, hf = wt >> 2;
+    const int t0 = lane & 3, t1 = lane >> 2;
+    const int lane0 = quarter * 32 + hf * 16;
+    const uint32_t lane_addr = static_cast<uint32_t>(lane0) << 16;
+    const uint32_t s_addr = tmem_base + lane_addr + t * kBN;
+    const uint32_t p_addr = tmem_base + lane_addr + kColP + t * (kBN / 2);
+    const uint32_t o_addr = tmem_base + lane_addr + kColO + t * D;
+    const int ntt = nt_tile[t];
+    int rr[2], pos[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      rr[e] = m_base + t * kBM + lane0 + t1 + 8 * e;  // row inside the sequence
+      pos[e] = rr[e] + off;                           // its position in key coordinates
+    }
+    const bool tracer = wt == 0 && lane == 0;
+    float slope_log2 = 0.f;
+    if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
+    float m_ref[2] = {neg_inf(), neg_inf()};  // reference max per row (log2 units)
+    float l_sum[2] = {0.f, 0.f};              // this thread's part of each row sum
+    bool ok = true;
+    int nc = 0;
+    for (int j = 0; j < ntt; ++j) {
+      if constexpr (SPARSE) {
+        if (!uses(t, j)) continue;
+      } else {
+        nc = j;
+      }
+      if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
+      int n0 = j * kBN, kfirst = 0;
+      if constexpr (kCache) {
+        const KeyTile kt = key_tile(j);
+        n0 = kt.pos;
+        kfirst = kt.lo;
+      }
+      int limit[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        limit[e] = k_len - n0;
+        if (kCausal) limit[e] = min(limit[e], pos[e] + 1 - n0);
+      }
+      const bool masked = __any_sync(0xffffffffu, limit[0] < kBN || limit[1] < kBN) ||
+                          (kCache && kfirst > 0);
+      auto hidden = [&](int col, int e) -> bool {
+        if constexpr (kCache) return col >= limit[e] || col < kfirst;
+        return col >= limit[e];
+      };
+      tc_fence_after();
+      uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+      tmem_ld16x256_x16_wait(s_addr, sr);
+      tc_fence_before();
+      mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+
+      // ---- pass 1: row maxima (log2 units) --------------------------------------
+      float mx[2] = {neg_inf(), neg_inf()};
+      if constexpr (ALIBI) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int col = 8 * k + 2 * t0 + c, idx = 4 * k + 2 * e + c;
+              float y = fmaf(__uint_as_float(sr[idx]), a.scale_log2,
+                             -slope_log2 * fabsf(static_cast<float>(n0 + col - pos[e])));
+              if (masked && hidden(col, e)) y = neg_inf();
+              sr[idx] = __float_as_uint(y);
+              mx[e] = fmaxf(mx[e], y);
+            }
+      } else if (!masked) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            mx[e] = max3(mx[e], __uint_as_float(sr[4 * k + 2 * e]),
+                         __uint_as_float(sr[4 * k + 2 * e + 1]));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              if (!hidden(8 * k + 2 * t0 + c, e))
+                mx[e] = fmaxf(mx[e], __uint_as_float(sr[4 * k + 2 * e + c]));
+      }
+      float alpha[2], nsub[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float pm = mx[e];
+        if constexpr (!ALIBI) pm = (pm == neg_inf()) ? pm : pm * a.scale_log2;
+        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
+        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
+        float m_use = m_ref[e];
+        if (pm > m_ref[e] + kTau) m_use = pm;  // also taken when m_ref is -inf
+        alpha[e] = (m_use == m_ref[e]) ? 1.f : ex2(m_ref[e] - m_use);
+        m_ref[e] = m_use;
+        nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
+      }
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
+
+      // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
+      uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
+      f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
+      const f2 scale2 = {a.scale_log2, a.scale_log2};
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
+          const f2 ns = {nsub[e], nsub[e]};
+          const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);
+          f2 p = {ex2(y.x), ex2(y.y)};
+          if (!ALIBI && masked) {
+            if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
+            if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
+          }
+          ps[e] = add2(ps[e], p);
+          pk[2 * k + e] = pack2<BF16>(p.x, p.y);
+        }
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+      // P_t is still being read by P.V of the previous key tile.
+      if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      tmem_st16x128_x16(p_addr, pk);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
+      // Rescale the output rows whose reference max moved.
+      if (nc > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
+        uint32_t o[32];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+        tmem_ld16x256_x8_wait(o_addr, o);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
+        tmem_st16x256_x8(o_addr, o);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[t]);
+      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
+      ++nc;
+    }
+    if constexpr (!SPARSE) nc = ntt;
+
+    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
+    if (ok && nc > 0) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      float l_tot[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        l_tot[e] = l_sum[e] + __shfl_xor_sync(0xffffffffu, l_sum[e], 1);
+        l_tot[e] += __shfl_xor_sync(0xffffffffu, l_tot[e], 2);
+      }
+      uint32_t o[32];
+      if (nc > 0) {
+        tmem_ld16x256_x8_wait(o_addr, o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (rr[e] >= q_len) continue;
+        const float inv_l = l_tot[e] > 0.f ? 1.f / l_tot[e] : 0.f;
+        uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
+                        2 * (bidx * a.o_sb + static_cast<long long>(q0 + rr[e]) * a.o_sm +
+                             h * a.o_sh + 2 * t0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint32_t*>(orow + 16 * k) =
+              pack2<BF16>(__uint_as_float(o[4 * k + 2 * e]) * inv_l,
+                          __uint_as_float(o[4 * k + 2 * e + 1]) * inv_l);
+        if (t0 == 0 && a.lse != nullptr) {
+          const float lse = l_tot[e] > 0.f ? (m_ref[e] + __log2f(l_tot[e])) * kLn2 : neg_inf();
+          a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + rr[e]] = lse;
+        }
+      }
+    }
+  } else {
     // Two threads per row: `half` 0 owns score columns 0..63 of each key tile
     // and output columns 0..D/2-1, `half` 1 the rest.  The two threads of a row
     // (same lane in warps w and w+4) exchange partial row maxima every tile and
@@ -548,14 +743,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(s_addr, sr[0]);
-      tmem_ld32(s_addr + 32, sr[1]);
 
       // Keys this row may see in the tile: columns [0, limit).  Tiles that need
       // no masking for any row of the warp take the unmasked path (warp-uniform).
       // Cache mode: columns before kfirst were seen by an earlier tile.
+      // (Computed before the TMEM loads: nothing runs between a load and its wait.)
       int n0 = j * kBN, kfirst = 0;
       if constexpr (kCache) {
         const KeyTile kt = key_tile(j);
@@ -571,6 +763,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return c0 + i >= limit;
       };
       const float dpos0 = static_cast<float>(n0 + c0 - pos_i);  // ALiBi distance of column c0
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(s_addr, sr[0]);
+      tmem_ld32(s_addr + 32, sr[1]);
       tmem_ld_wait(sr[0]);
       tmem_ld_wait(sr[1]);
       if constexpr (kSepP) {  // S_t may now be overwritten by the next Q.K^T
@@ -730,6 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + r] = lse;
       }
     }
+  }
   }
 
   tc_fence_before();
