@@ -141,3 +141,18 @@ def test_full_size_sampled(mea, orc):
         assert_lse_close(lse[b], rl[0], f"{c.name} b={b}")
         p = c.past[b]
         assert np.array_equal(kc[b, p:p + c.M].cpu().to(torch.float64).numpy(), rkc[0, p:p + c.M])
+
+
+@pytest.mark.parametrize("causal,alibi", [(False, False), (True, False), (True, True)])
+def test_chunk_repeatable(mea, causal, alibi):
+    """Ten launches on the same input give bit-identical outputs (a race between
+    a TMEM load and its use would show as run-to-run differences)."""
+    c = synth.make_chunk("chunk_rep", [0, 1, 128, 200, 1000], 300, 1400, 4, 2, 64, "f16", causal,
+                         seed=450, alibi=alibi)
+    first = None
+    for _ in range(10):
+        out, lse, _, _ = _run(mea, c)
+        if first is None:
+            first = (out, lse)
+        else:
+            assert torch.equal(out, first[0]) and torch.equal(lse, first[1])

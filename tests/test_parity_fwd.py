@@ -195,3 +195,14 @@ def test_gqa_alibi_full_size_sampled(mea, orc):
     rows = _sample_rows(np.random.default_rng(4), p.B, p.M, p.Hq, n=256,
                         edges=(0, 1, 127, 128, 255, 256, 2048, 4095))
     _check_sampled(mea, orc, p, rows)
+
+
+@pytest.mark.parametrize("K,dtype,bias", [(64, "f16", "none"), (64, "f16", "causal"),
+                                          (128, "bf16", "causal")])
+def test_repeatable_each_layout(mea, K, dtype, bias):
+    """Both TMEM layouts give bit-identical results over repeated launches."""
+    p = synth.make_prefill("rep_layout", 2, 700, 650, 4, 2, K, dtype, bias, seed=81)
+    first = _run_gpu(mea, p)
+    for _ in range(5):
+        again = _run_gpu(mea, p)
+        assert torch.equal(again[0], first[0]) and torch.equal(again[1], first[1])
