@@ -11,12 +11,13 @@
 //
 // CTA organisation (608 threads, one CTA per SM):
 //   warps 0-7   softmax / rescale / epilogue for query tile 0 (TMEM lanes 0-127):
-//               two threads per row, warps 0-3 on score columns 0-63 and the
-//               first half of the output row, warps 4-7 on the other halves
+//               each warp on 16 lanes of its lane quarter, four threads per row
+//               (a quarter of the columns each) in one warp
 //   warps 8-15  the same for query tile 1 (rows +128)
-//   warp  16    TMEM allocator; one thread issues every MMA of query tile 0
-//   warp  17    one thread issues every MMA of query tile 1 (the two tiles do not
-//               wait for each other: each follows its own softmax)
+//   warp  16    TMEM allocator; one thread issues every MMA of query tile 0 (and,
+//               with P written over S, of query tile 1 too, interleaved)
+//   warp  17    separate-P layout: one thread issues every MMA of query tile 1
+//               (the two tiles do not wait for each other)
 //   warp  18    the single TMA-issuing thread
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
 // current key tile; P = exp(S - m) as 16-bit pairs is written back over S, each
@@ -41,7 +42,7 @@ constexpr int kBN = 128;        // keys per tile
 constexpr int kThreads = 608;
 constexpr int kMmaWarp = 16;   // + tile: warps 16 and 17 each issue one query tile's MMAs
 constexpr int kTmaWarp = 18;
-constexpr int kSoftmaxThreadsPerTile = 256;  // two threads per row
+constexpr int kSoftmaxThreadsPerTile = 256;  // four threads per row
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceeds it by < 2^8
 constexpr float kLog2e = 1.4426950408889634f;
@@ -56,11 +57,8 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kKV = 2 * kTileBytes;
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1 + 8 + 2;
-  // Row-pair exchange: partial maxima [tile][parity][half][row], sums [tile][half][row].
-  static constexpr int kXMax = kBar + kNumBars * 8;
-  static constexpr int kXSum = kXMax + 2 * 2 * 2 * kBM * 4;
-  static constexpr int kTmemSlot = kXSum + 2 * 2 * kBM * 4;
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1 + 2;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
 };
@@ -132,10 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_ready = s_full + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* mma_done = o_done + 2;
-  uint64_t* pair_bar = mma_done + 1;  // [tile][lane quarter]: the two warps of a row pair
-  uint64_t* s_free = pair_bar + 8;    // S_t read out by the softmax (separate-P layout)
-  float* xmax = reinterpret_cast<float*>(smem + L::kXMax);
-  float* xsum = reinterpret_cast<float*>(smem + L::kXSum);
+  uint64_t* s_free = mma_done + 1;    // S_t read out by the softmax (separate-P layout)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
@@ -276,7 +271,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_done, kSepP ? 2 : 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 64);
     for (int t = 0; t < 2; ++t) mbar_init(&s_free[t], kSoftmaxThreadsPerTile);
     *abort_flag = 0;
     fence_barrier_init();
@@ -510,22 +504,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================== softmax warpgroups ===============================
-  if constexpr (kSepP) {
-    // Separate-P layout (K = 64, fp16): eight warps per query tile, each on 16
-    // TMEM lanes of its lane quarter (16x256b shape); a thread holds rows
-    // lane0 + t1 and lane0 + t1 + 8 and, of each 8-column group, the columns
-    // 2 t0 and 2 t0 + 1 (t0 = lane % 4, t1 = lane / 4).  The four threads of a
-    // row are lanes 4 t1 .. 4 t1 + 3 of one warp: row maxima and row sums
-    // combine with two shuffles.  P goes back as 16-bit pairs with the 16x128b
-    // shape, which puts keys 8k + 2 t0, 8k + 2 t0 + 1 into column 4k + t0.
+    // Eight warps per query tile, each on 16 TMEM lanes of its lane quarter
+    // (16-lane shapes): a thread holds rows lane0 + t1 and lane0 + t1 + 8 and, of
+    // every 8-column group, the columns 2 t0 and 2 t0 + 1 (t0 = lane % 4,
+    // t1 = lane / 4).  The four threads of a row are lanes 4 t1 .. 4 t1 + 3 of
+    // one warp, so row maxima and row sums combine with two shuffles.  P goes
+    // back as 16-bit pairs with the 16x128b shape, which puts keys 8k + 2 t0,
+    // 8k + 2 t0 + 1 into column 4k + t0 of the packed block that the P.V MMA
+    // reads: the separate P columns, or (P over S) each 32-key chunk's first 16
+    // S columns, with bf16's P - P_hi in the chunk's last 16.
     const int t = warp >> 3;
     const int wt = warp & 7, quarter = wt & 3, hf = wt >> 2;
     const int t0 = lane & 3, t1 = lane >> 2;
     const int lane0 = quarter * 32 + hf * 16;
     const uint32_t lane_addr = static_cast<uint32_t>(lane0) << 16;
     const uint32_t s_addr = tmem_base + lane_addr + t * kBN;
-    const uint32_t p_addr = tmem_base + lane_addr + kColP + t * (kBN / 2);
+    const uint32_t p_addr = tmem_base + lane_addr + kColP + t * (kSepP ? kBN / 2 : kBN);
     const uint32_t o_addr = tmem_base + lane_addr + kColO + t * D;
+    constexpr int kOReg = D / 2;  // O registers of a thread: 2 rows x D/4 columns
+    auto ld_o = [&](uint32_t(&o)[kOReg]) {
+      if constexpr (D == 64) tmem_ld16x256_x8_wait(o_addr, o);
+      else tmem_ld16x256_x16_wait(o_addr, o);
+    };
+    auto st_o = [&](const uint32_t(&o)[kOReg]) {
+      if constexpr (D == 64) tmem_st16x256_x8(o_addr, o);
+      else tmem_st16x256_x16(o_addr, o);
+    };
     const int ntt = nt_tile[t];
     int rr[2], pos[2];
 #pragma unroll
@@ -548,6 +552,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
+      // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
+      // need no masking for any row of the warp take the unmasked path.
       int n0 = j * kBN, kfirst = 0;
       if constexpr (kCache) {
         const KeyTile kt = key_tile(j);
@@ -569,10 +575,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
       tmem_ld16x256_x16_wait(s_addr, sr);
-      tc_fence_before();
-      mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+      if constexpr (kSepP) {
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+      }
 
       // ---- pass 1: row maxima (log2 units) --------------------------------------
+      // ALiBi: the bias of column 8k + 2 t0 + c in row e is -slope |db[e] + 8k + c|,
+      // recomputed in both passes (cheaper than keeping the biased logits live).
+      // Under a causal mask a visible key is never after the query, so the bias
+      // is linear in the column there: slope (db[e] + 8k + c); hidden columns are
+      // set to -inf anyway.
+      float db[2], sdb[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        db[e] = static_cast<float>(n0 + 2 * t0 - pos[e]);
+        sdb[e] = slope_log2 * db[e];
+      }
+      auto bias = [&](int k, int c, int e) -> float {
+        if constexpr (kCausal) return fmaf(slope_log2, static_cast<float>(8 * k + c), sdb[e]);
+        return -slope_log2 * fabsf(db[e] + static_cast<float>(8 * k + c));
+      };
       float mx[2] = {neg_inf(), neg_inf()};
       if constexpr (ALIBI) {
 #pragma unroll
@@ -581,11 +604,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 2; ++e)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const int col = 8 * k + 2 * t0 + c, idx = 4 * k + 2 * e + c;
-              float y = fmaf(__uint_as_float(sr[idx]), a.scale_log2,
-                             -slope_log2 * fabsf(static_cast<float>(n0 + col - pos[e])));
-              if (masked && hidden(col, e)) y = neg_inf();
-              sr[idx] = __float_as_uint(y);
+              float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), a.scale_log2, bias(k, c, e));
+              if (masked && hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
+              sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
               mx[e] = fmaxf(mx[e], y);
             }
       } else if (!masked) {
@@ -621,45 +642,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
 
       // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
-      uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
       f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
       const f2 scale2 = {a.scale_log2, a.scale_log2};
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
-          const f2 ns = {nsub[e], nsub[e]};
-          const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);
-          f2 p = {ex2(y.x), ex2(y.y)};
-          if (!ALIBI && masked) {
-            if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
-            if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
-          }
-          ps[e] = add2(ps[e], p);
-          pk[2 * k + e] = pack2<BF16>(p.x, p.y);
+      auto p_pair = [&](int k, int e) -> f2 {
+        const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
+        const f2 ns = {nsub[e], nsub[e]};
+        const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
+        f2 p = {ex2(y.x), ex2(y.y)};
+        if (!ALIBI && masked) {
+          if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
+          if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
         }
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-      // P_t is still being read by P.V of the previous key tile.
-      if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
-      tc_fence_after();
-      tmem_st16x128_x16(p_addr, pk);
+        ps[e] = add2(ps[e], p);
+        return p;
+      };
+      if constexpr (kSepP) {
+        uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const f2 p = p_pair(k, e);
+            pk[2 * k + e] = pack2<BF16>(p.x, p.y);
+          }
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+        // P_t is still being read by P.V of the previous key tile.
+        if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)))
+          break;
+        tc_fence_after();
+        tmem_st16x128_x16(p_addr, pk);
+      } else {
+        // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
+        // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
+        // lo pairs repetitions 4..7.
+#pragma unroll
+        for (int C = 0; C < 4; ++C) {
+          uint32_t pc[kSplitP ? 16 : 8];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const f2 p = p_pair(4 * C + kk, e);
+              const uint32_t hi = pack2<BF16>(p.x, p.y);
+              pc[2 * kk + e] = hi;
+              if constexpr (kSplitP) {
+                const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
+                const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
+                pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
+              }
+            }
+          if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
+          else tmem_st16x128_x4(p_addr + 32 * C, pc);
+        }
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+      }
 #pragma unroll
       for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
-      // Rescale the output rows whose reference max moved.
+      // Rescale the output rows whose reference max moved (after the previous
+      // P.V has written O).
       if (nc > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
         if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
-        uint32_t o[32];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
-        tmem_ld16x256_x8_wait(o_addr, o);
+        if constexpr (!kSepP) {
+          if (!(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+        }
+        uint32_t o[kOReg];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+        ld_o(o);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < D / 8; ++k)
 #pragma unroll
           for (int e = 0; e < 2; ++e)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
               o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
-        tmem_st16x256_x8(o_addr, o);
+        st_o(o);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -679,12 +736,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_tot[e] = l_sum[e] + __shfl_xor_sync(0xffffffffu, l_sum[e], 1);
         l_tot[e] += __shfl_xor_sync(0xffffffffu, l_tot[e], 2);
       }
-      uint32_t o[32];
+      uint32_t o[kOReg];
       if (nc > 0) {
-        tmem_ld16x256_x8_wait(o_addr, o);
+        ld_o(o);
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
+        for (int i = 0; i < kOReg; ++i) o[i] = 0u;
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -694,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         2 * (bidx * a.o_sb + static_cast<long long>(q0 + rr[e]) * a.o_sm +
                              h * a.o_sh + 2 * t0);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < D / 8; ++k)
           *reinterpret_cast<uint32_t*>(orow + 16 * k) =
               pack2<BF16>(__uint_as_float(o[4 * k + 2 * e]) * inv_l,
                           __uint_as_float(o[4 * k + 2 * e + 1]) * inv_l);
@@ -704,229 +761,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
-    // Two threads per row: `half` 0 owns score columns 0..63 of each key tile
-    // and output columns 0..D/2-1, `half` 1 the rest.  The two threads of a row
-    // (same lane in warps w and w+4) exchange partial row maxima every tile and
-    // partial row sums at the end through shared memory, ordered by an
-    // mbarrier of 64 arrivals (`pair_bar`), so both apply the same reference max.
-    const int t = warp >> 3;                   // query tile
-    const int half = (warp >> 2) & 1;          // column half
-    const int wq = warp & 3;                   // TMEM lane quarter
-    const int row = wq * 32 + lane;            // row inside the tile
-    const int r = m_base + t * kBM + row;      // row inside the sequence
-    const int pos_i = r + off;                 // its position in key coordinates
-    const int ntt = nt_tile[t];
-    const int c0 = half * (kBN / 2);           // first score column of this thread
-    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t s_addr = tmem_base + lane_addr + t * kBN + c0;
-    const uint32_t o_addr = tmem_base + lane_addr + kColO + t * D + half * (D / 2);
-    // Where this thread's P goes: its own columns (separate-P layout, 16 packed
-    // columns per 32 keys) or over its S columns (32 per 32 keys, hi then lo).
-    const uint32_t p_addr = kSepP ? tmem_base + lane_addr + kColP + t * (kBN / 2) + half * (kBN / 4)
-                                  : s_addr;
-    uint64_t* pbar = &pair_bar[t * 4 + wq];
-    const bool tracer = (warp & 7) == 0 && lane == 0;
-    float slope_log2 = 0.f;
-    if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
-
-    float m_ref = neg_inf();  // reference max (log2 units) used for the exponentials
-    float l_sum = 0.f;        // this thread's part of the running sum of 2^(x - m_ref)
-    bool ok = true;
-
-    int nc = 0;  // key tiles this query tile has computed (its barrier phases)
-    for (int j = 0; j < ntt; ++j) {
-      if constexpr (SPARSE) {
-        if (!uses(t, j)) continue;
-      } else {
-        nc = j;  // dense: every key tile up to ntt is computed
-      }
-      if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
-
-      // Keys this row may see in the tile: columns [0, limit).  Tiles that need
-      // no masking for any row of the warp take the unmasked path (warp-uniform).
-      // Cache mode: columns before kfirst were seen by an earlier tile.
-      // (Computed before the TMEM loads: nothing runs between a load and its wait.)
-      int n0 = j * kBN, kfirst = 0;
-      if constexpr (kCache) {
-        const KeyTile kt = key_tile(j);
-        n0 = kt.pos;
-        kfirst = kt.lo;
-      }
-      int limit = k_len - n0;
-      if (kCausal) limit = min(limit, pos_i + 1 - n0);
-      const bool masked = __any_sync(0xffffffffu, limit < kBN) || (kCache && kfirst > 0);
-      // Column i of this thread is outside [kfirst, limit).
-      auto hidden = [&](int i) -> bool {
-        if constexpr (kCache) return c0 + i >= limit || c0 + i < kfirst;
-        return c0 + i >= limit;
-      };
-      const float dpos0 = static_cast<float>(n0 + c0 - pos_i);  // ALiBi distance of column c0
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(s_addr, sr[0]);
-      tmem_ld32(s_addr + 32, sr[1]);
-      tmem_ld_wait(sr[0]);
-      tmem_ld_wait(sr[1]);
-      if constexpr (kSepP) {  // S_t may now be overwritten by the next Q.K^T
-        tc_fence_before();
-        mbar_arrive(&s_free[t]);
-      }
-
-      // ---- pass 1: partial row max (log2 units) ------------------------------
-      // Without ALiBi the max is taken on the raw scores (scale >= 0) and scaled
-      // once; with ALiBi the biased logit is formed here, in place.
-      float mx[4] = {neg_inf(), neg_inf(), neg_inf(), neg_inf()};
-      if constexpr (ALIBI) {
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
-          float y = fmaf(__uint_as_float(sr[i >> 5][i & 31]), a.scale_log2,
-                         -slope_log2 * fabsf(dpos0 + static_cast<float>(i)));
-          if (masked && hidden(i)) y = neg_inf();
-          sr[i >> 5][i & 31] = __float_as_uint(y);
-          mx[i & 3] = fmaxf(mx[i & 3], y);
-        }
-      } else if (!masked) {
-#pragma unroll
-        for (int i = 0; i < kBN / 2; i += 2)
-          mx[(i >> 1) & 3] = max3(mx[(i >> 1) & 3], __uint_as_float(sr[i >> 5][i & 31]),
-                                  __uint_as_float(sr[i >> 5][(i + 1) & 31]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < kBN / 2; ++i)
-          if (!hidden(i)) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i >> 5][i & 31]));
-      }
-      float pmax = max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      if constexpr (!ALIBI) pmax = (pmax == neg_inf()) ? pmax : pmax * a.scale_log2;
-
-      // ---- exchange with the other half of the row -----------------------------
-      float* xm = xmax + ((t * 2 + (nc & 1)) * 2) * kBM;
-      xm[half * kBM + row] = pmax;
-      mbar_arrive(pbar);
-      if (!(ok = mbar_wait_warp(pbar, nc & 1, abort_flag, a.status))) break;
-      const float tmax = fmaxf(pmax, xm[(1 - half) * kBM + row]);
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
-      float m_use = m_ref;
-      if (tmax > m_ref + kTau) m_use = tmax;  // also taken when m_ref is -inf
-      const float alpha = (m_use == m_ref) ? 1.f : ex2(m_ref - m_use);
-      m_ref = m_use;
-      const float nsub = (m_use == neg_inf()) ? 0.f : -m_use;
-
-      // ---- pass 2: P = 2^(logit - m) in place, partial row sums ----------------
-      f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
-      const f2 scale2 = {a.scale_log2, a.scale_log2}, nsub2 = {nsub, nsub};
-#pragma unroll
-      for (int i = 0; i < kBN / 2; i += 2) {
-        const f2 v = {__uint_as_float(sr[i >> 5][i & 31]),
-                      __uint_as_float(sr[i >> 5][(i + 1) & 31])};
-        const f2 y = ALIBI ? add2(v, nsub2) : fma2(v, scale2, nsub2);
-        f2 p = {ex2(y.x), ex2(y.y)};
-        if (!ALIBI && masked) {
-          if (hidden(i)) p.x = 0.f;
-          if (hidden(i + 1)) p.y = 0.f;
-        }
-        ps[(i >> 1) & 1] = add2(ps[(i >> 1) & 1], p);
-        sr[i >> 5][i & 31] = __float_as_uint(p.x);
-        sr[i >> 5][(i + 1) & 31] = __float_as_uint(p.y);
-      }
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-      if constexpr (kSepP) {  // P_t is still being read by P.V of the previous tile
-        if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-      }
-      // Store P as 16-bit pairs over each 32-key chunk's own S columns (keys
-      // 32C..32C+31 -> columns 32C..32C+15).  With bf16 (8 significant bits) P
-      // is stored as hi + lo, the low part P - P_hi in columns 32C+16..32C+31,
-      // so that P.V carries ~16 bits of P.
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const f2 p = {__uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1])};
-          pk[i] = pack2<BF16>(p.x, p.y);
-          if constexpr (kSplitP) {
-            const f2 hi = {__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u)};
-            const f2 res = fma2(hi, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
-            lo[i] = pack2<BF16>(res.x, res.y);
-          }
-        }
-        tmem_st16(p_addr + c * (kSepP ? 16 : 32), pk);
-        if constexpr (kSplitP) tmem_st16(p_addr + c * 32 + 16, lo);
-      }
-      const f2 pst = add2(ps[0], ps[1]);
-      l_sum = l_sum * alpha + (pst.x + pst.y);
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
-
-      // Rescale this thread's half of the output accumulator when the row's
-      // reference max moved.
-      if (nc > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
-        if (!(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(o_addr + c * 32, o);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_ready[t]);
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
-      ++nc;
-    }
-
-    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
-    if constexpr (!SPARSE) nc = ntt;
-    if (ok && nc > 0) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
-    if (ok) {
-      // Row sum = both halves' parts (same reference max).
-      xsum[(t * 2 + half) * kBM + row] = l_sum;
-      mbar_arrive(pbar);
-      ok = mbar_wait_warp(pbar, nc & 1, abort_flag, a.status);
-    }
-    if (ok) {
-      const float l_tot = l_sum + xsum[(t * 2 + 1 - half) * kBM + row];
-      tc_fence_after();
-      const bool valid = r < q_len;
-      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
-                      2 * (bidx * a.o_sb + static_cast<long long>(q0 + r) * a.o_sm + h * a.o_sh +
-                           half * (D / 2));
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o[32];
-        if (nc > 0) {
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
-                              __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
-      }
-      if (valid && half == 0 && a.lse != nullptr) {
-        const float lse = l_tot > 0.f ? (m_ref + __log2f(l_tot)) * kLn2 : neg_inf();
-        a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + r] = lse;
-      }
-    }
-  }
   }
 
   tc_fence_before();
