@@ -526,7 +526,7 @@ def measure_backward(mea, p, dev, stream, tc_peak, iters=5):
     tf = f / (ms * 1e-3) / 1e12
     return {"workload": "bwd_" + p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
             "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor",
-            "kernel": "mma.sync m16n8k16 (legacy tensor path)"}
+            "kernel": "bwd_kernel (tcgen05, TMA; dq by TMA tensor reductions)"}
 
 
 def measure_decode(mea, d, dev, stream, hbm_peak, iters=20):
