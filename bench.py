@@ -548,13 +548,16 @@ def measure_decode(mea, d, dev, stream, hbm_peak, iters=20):
 # ---------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on the host cores, bounded sample
 # ---------------------------------------------------------------------------
+_F64_INPUTS = {}
+
+
 def cpu_baseline(p: synth.Prefill, seconds: float):
     import oracle
 
     orc = oracle.get()
-    qf = p.q.to(torch.float64).numpy()
-    kf = p.k.to(torch.float64).numpy()
-    vf = p.v.to(torch.float64).numpy()
+    if p.name not in _F64_INPUTS:  # exact fp64 copies, made once per workload
+        _F64_INPUTS[p.name] = tuple(t.to(torch.float64).numpy() for t in (p.q, p.k, p.v))
+    qf, kf, vf = _F64_INPUTS[p.name]
     rng = np.random.default_rng(0)
     rows_done, t_used, batch = 0, 0.0, 64
     while t_used < seconds:
@@ -578,7 +581,8 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     p = synth.noncausal_sweep(4096)
-    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    # About two minutes of oracle work in all, whatever --steps / --warmup are.
+    per_step = max(0.05, min(15.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(p, per_step / 4)
     t_start = time.perf_counter()
