@@ -83,3 +83,30 @@ def test_bwd_varlen(mea, causal):
     p = synth.make_varlen(f"bwd_varlen_c{causal}", [1, 63, 64, 65, 200, 0, 130], 4, 2, 128, "bf16",
                           causal, seed=230, alibi=causal)
     _check(mea, p)
+
+
+@pytest.mark.parametrize("case", ["noncausal_b8_h16_m2048_k64_f16", "gqa_alibi_causal_b4_m4096"])
+def test_bwd_full_size_properties(mea, case):
+    """The benchmarked backward workloads, at full size, through properties that
+    hold for every row: its weights sum to one, so per (batch, kv head) the keys'
+    dv sum to the rows' dout summed over the head group; each row of dS sums to
+    zero, so the keys' dk sum to zero.  Tolerance: the 16-bit rounding of each
+    gradient element (relative 2^-9 bf16, 2^-12 fp16), against the sum of
+    magnitudes."""
+    p = synth.noncausal_sweep(2048) if case.startswith("noncausal") else synth.gqa_alibi_causal()
+    dout = synth.randn(tuple(p.q.shape), p.dtype, synth.generator(p.seed + 17)).to(DEV)
+    q, k, v = p.q.to(DEV), p.k.to(DEV), p.v.to(DEV)
+    out, lse = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi)
+    dq, dk, dv = mea.mea_bwd(q, k, v, out, dout, lse, bias=p.bias, scale=p.scale, alibi=p.alibi)
+    torch.cuda.synchronize()
+    assert mea.read_device_status() == 0
+    for g in (dq, dk, dv):
+        assert torch.isfinite(g).all()
+    G = p.Hq // p.Hkv
+    rel = 4e-3 if p.dtype == "bf16" else 5e-4
+    sdv = dv.double().sum(dim=1)
+    sdo = dout.double().view(p.B, p.M, p.Hkv, G, p.K).sum(dim=(1, 3))
+    mag = dv.double().abs().sum(dim=1) + dout.double().abs().view(p.B, p.M, p.Hkv, G, p.K).sum(dim=(1, 3))
+    assert ((sdv - sdo).abs() <= rel * mag + 1e-6).all(), (sdv - sdo).abs().max().item()
+    sdk = dk.double().sum(dim=1)
+    assert (sdk.abs() <= rel * dk.double().abs().sum(dim=1) + 1e-6).all(), sdk.abs().max().item()
