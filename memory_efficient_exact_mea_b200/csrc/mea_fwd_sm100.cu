@@ -30,6 +30,8 @@
 // 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
 
+#include <type_traits>
+
 #include "mea_internal.h"
 #include "sm100.cuh"
 
@@ -598,17 +600,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       float mx[2] = {neg_inf(), neg_inf()};
       if constexpr (ALIBI) {
+        auto biased = [&](auto msk) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
+          for (int k = 0; k < 16; ++k)
 #pragma unroll
-          for (int e = 0; e < 2; ++e)
+            for (int e = 0; e < 2; ++e)
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), a.scale_log2, bias(k, c, e));
-              if (masked && hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
-              sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
-              mx[e] = fmaxf(mx[e], y);
-            }
+              for (int c = 0; c < 2; ++c) {
+                float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), a.scale_log2, bias(k, c, e));
+                if constexpr (decltype(msk)::value) {
+                  if (hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
+                }
+                sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
+                mx[e] = fmaxf(mx[e], y);
+              }
+        };
+        if (masked) biased(std::true_type{});
+        else biased(std::false_type{});
       } else if (!masked) {
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -642,60 +650,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
 
       // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
+      // Instantiated separately for tiles with and without masking, so the
+      // per-element mask tests exist only in the masked copy (ALiBi's masked
+      // logits are already -inf, so its P needs none).
       f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
       const f2 scale2 = {a.scale_log2, a.scale_log2};
-      auto p_pair = [&](int k, int e) -> f2 {
-        const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
-        const f2 ns = {nsub[e], nsub[e]};
-        const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
-        f2 p = {ex2(y.x), ex2(y.y)};
-        if (!ALIBI && masked) {
-          if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
-          if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
-        }
-        ps[e] = add2(ps[e], p);
-        return p;
-      };
-      if constexpr (kSepP) {
-        uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const f2 p = p_pair(k, e);
-            pk[2 * k + e] = pack2<BF16>(p.x, p.y);
+      auto pass2 = [&](auto msk) -> bool {
+        constexpr bool kMsk = !ALIBI && decltype(msk)::value;
+        auto p_pair = [&](int k, int e) -> f2 {
+          const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
+          const f2 ns = {nsub[e], nsub[e]};
+          const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
+          f2 p = {ex2(y.x), ex2(y.y)};
+          if constexpr (kMsk) {
+            if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
+            if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
           }
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-        // P_t is still being read by P.V of the previous key tile.
-        if (nc > 0 && !(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)))
-          break;
-        tc_fence_after();
-        tmem_st16x128_x16(p_addr, pk);
-      } else {
-        // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
-        // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
-        // lo pairs repetitions 4..7.
+          ps[e] = add2(ps[e], p);
+          return p;
+        };
+        if constexpr (kSepP) {
+          uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
 #pragma unroll
-        for (int C = 0; C < 4; ++C) {
-          uint32_t pc[kSplitP ? 16 : 8];
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
+          for (int k = 0; k < 16; ++k)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const f2 p = p_pair(4 * C + kk, e);
-              const uint32_t hi = pack2<BF16>(p.x, p.y);
-              pc[2 * kk + e] = hi;
-              if constexpr (kSplitP) {
-                const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
-                const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
-                pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
-              }
+              const f2 p = p_pair(k, e);
+              pk[2 * k + e] = pack2<BF16>(p.x, p.y);
             }
-          if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
-          else tmem_st16x128_x4(p_addr + 32 * C, pc);
+          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+          // P_t is still being read by P.V of the previous key tile.
+          if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
+            return false;
+          tc_fence_after();
+          tmem_st16x128_x16(p_addr, pk);
+        } else {
+          // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
+          // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
+          // lo pairs repetitions 4..7.
+#pragma unroll
+          for (int C = 0; C < 4; ++C) {
+            uint32_t pc[kSplitP ? 16 : 8];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const f2 p = p_pair(4 * C + kk, e);
+                const uint32_t hi = pack2<BF16>(p.x, p.y);
+                pc[2 * kk + e] = hi;
+                if constexpr (kSplitP) {
+                  const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
+                  const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
+                  pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
+                }
+              }
+            if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
+            else tmem_st16x128_x4(p_addr + 32 * C, pc);
+          }
+          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
         }
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-      }
+        return true;
+      };
+      if (!(ok = (!ALIBI && masked) ? pass2(std::true_type{}) : pass2(std::false_type{}))) break;
 #pragma unroll
       for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
