@@ -42,6 +42,8 @@
 
 #include <algorithm>
 
+#include <type_traits>
+
 #include "mea_internal.h"
 #include "sm100.cuh"
 
@@ -436,58 +438,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* nd = s_delta + slot * BM + c0;
       uint8_t* ds_buf = ds_row + (s & 1) * C::kDSTile;
       uint32_t pk[kCols / 2];
-      // 32 columns at a time: read S^T, dP^T out of TMEM (releasing them after the
-      // last chunk), then P = 2^(s*scale*log2e - lse*log2e) and dS = P (dP - D).
+      // K = 128: instantiated for blocks with and without per-element masks, so
+      // the unmasked copy carries no mask arithmetic (`full` depends on the warp
+      // only, through c0, as the warp-collective TMEM loads inside require).
+      // K = 64: one copy with a run-time test (two copies spill there).
+      auto p_ds = [&](auto msk) {
+        // 32 columns at a time: read S^T, dP^T out of TMEM (releasing them after the
+        // last chunk), then P = 2^(s*scale*log2e - lse*log2e) and dS = P (dP - D).
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c) {
-        uint32_t sr[32], dr[32], dk[16];
-        tmem_ld32(tS + 32 * c, sr);
-        tmem_ld32(tDP + 32 * c, dr);
-        tmem_ld_wait(sr);
-        tmem_ld_wait(dr);
-        if (c == kCols / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(s_free);  // the next block's S^T / dP^T may be written now
-          if (tracer) BWD_TRACE(s, 9);
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int k = 32 * c + e;
-          const float2 l = *reinterpret_cast<const float2*>(nl + k);
-          const float2 dd = *reinterpret_cast<const float2*>(nd + k);
-          f2 x = fma2(f2{__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])}, scale2,
-                      f2{l.x, l.y});
-          const int pos = m0 + c0 + k + off;  // query position of column k, key coordinates
-          if constexpr (ALIBI) {
-            x.x -= slope_log2 * fabsf(static_cast<float>(pos - j_loc));
-            x.y -= slope_log2 * fabsf(static_cast<float>(pos + 1 - j_loc));
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t sr[32], dr[32], dk[16];
+          tmem_ld32(tS + 32 * c, sr);
+          tmem_ld32(tDP + 32 * c, dr);
+          tmem_ld_wait(sr);
+          tmem_ld_wait(dr);
+          if (c == kCols / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(s_free);  // the next block's S^T / dP^T may be written now
+            if (tracer) BWD_TRACE(s, 9);
           }
-          f2 p = {ex2(x.x), ex2(x.y)};
-          if (!full) {
-            bool v0 = key_ok, v1 = key_ok;
-            if constexpr (kCausal) {
-              v0 = v0 && j_loc <= pos;
-              v1 = v1 && j_loc <= pos + 1;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int k = 32 * c + e;
+            const float2 l = *reinterpret_cast<const float2*>(nl + k);
+            const float2 dd = *reinterpret_cast<const float2*>(nd + k);
+            f2 x = fma2(f2{__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])}, scale2,
+                        f2{l.x, l.y});
+            const int pos = m0 + c0 + k + off;  // query position of column k, key coordinates
+            if constexpr (ALIBI) {
+              x.x -= slope_log2 * fabsf(static_cast<float>(pos - j_loc));
+              x.y -= slope_log2 * fabsf(static_cast<float>(pos + 1 - j_loc));
             }
-            if (!v0) p.x = 0.f;
-            if (!v1) p.y = 0.f;
+            f2 p = {ex2(x.x), ex2(x.y)};
+            if (flag_on(msk)) {
+              bool v0 = key_ok, v1 = key_ok;
+              if constexpr (kCausal) {
+                v0 = v0 && j_loc <= pos;
+                v1 = v1 && j_loc <= pos + 1;
+              }
+              if (!v0) p.x = 0.f;
+              if (!v1) p.y = 0.f;
+            }
+            const f2 t = add2(f2{__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])},
+                              f2{dd.x, dd.y});
+            const f2 ds = fma2(p, t, zero2);
+            pk[k / 2] = pack2<BF16>(p.x, p.y);
+            dk[e / 2] = pack2<BF16>(ds.x, ds.y);
           }
-          const f2 t = add2(f2{__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])},
-                            f2{dd.x, dd.y});
-          const f2 ds = fma2(p, t, zero2);
-          pk[k / 2] = pack2<BF16>(p.x, p.y);
-          dk[e / 2] = pack2<BF16>(ds.x, ds.y);
-        }
-        // dS^T row `row`, columns c0+32c .. +31, in the 128-byte-swizzled layout the
-        // MMA descriptors read: 16-byte piece u of a 64-column chunk sits at u ^ (row & 7).
-        const int col = c0 + 32 * c;
-        const int plane = col >> 6;
+          // dS^T row `row`, columns c0+32c .. +31, in the 128-byte-swizzled layout the
+          // MMA descriptors read: 16-byte piece u of a 64-column chunk sits at u ^ (row & 7).
+          const int col = c0 + 32 * c;
+          const int plane = col >> 6;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int piece = ((col & 63) >> 3) + u;
-          *reinterpret_cast<uint4*>(ds_buf + plane * C::kKVChunk + ((piece ^ (row & 7)) << 4)) =
-              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          for (int u = 0; u < 4; ++u) {
+            const int piece = ((col & 63) >> 3) + u;
+            *reinterpret_cast<uint4*>(ds_buf + plane * C::kKVChunk + ((piece ^ (row & 7)) << 4)) =
+                make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+          }
         }
+      };
+      if constexpr (D == 128) {
+        if (full) p_ds(std::false_type{});
+        else p_ds(std::true_type{});
+      } else {
+        p_ds(!full);
       }
       if (tracer) BWD_TRACE(s, 10);
       // The previous block's dV MMAs still read P^T (queries 2c, 2c+1 in column c).

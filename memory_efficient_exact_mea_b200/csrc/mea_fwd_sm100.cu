@@ -115,6 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // = 512), so S_t is free as soon as the softmax has read it and the next
   // Q.K^T of the same tile runs during its softmax.  Otherwise P is written over S.
   constexpr bool kSepP = (D == 64) && !BF16;
+  // Softmax tile body specialised separately for masked and unmasked tiles.
+  constexpr bool kTileCopies = !ALIBI && MODE == kModeDense && !kPacked;
   constexpr uint32_t kColP = kSepP ? 2 * kBN : 0;          // + t * (kSepP ? kBN/2 : kBN)
   constexpr uint32_t kColO = kSepP ? 2 * kBN + kBN : 2 * kBN;  // + t * D
   constexpr int S = L::kSlots;
@@ -542,6 +544,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool tracer = wt == 0 && lane == 0;
     float slope_log2 = 0.f;
     if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
+    // A zero scale is taken as 1e-30 (the same softmax to fp32 precision for any
+    // finite score), so that -inf * scale stays -inf for hidden keys.
+    const float scale_log2 = fmaxf(a.scale_log2, 1e-30f);
     float m_ref[2] = {neg_inf(), neg_inf()};  // reference max per row (log2 units)
     float l_sum[2] = {0.f, 0.f};              // this thread's part of each row sum
     bool ok = true;
@@ -574,166 +579,179 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kCache) return col >= limit[e] || col < kfirst;
         return col >= limit[e];
       };
-      tc_fence_after();
-      uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
-      tmem_ld16x256_x16_wait(s_addr, sr);
-      if constexpr (kSepP) {
-        tc_fence_before();
-        mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
-      }
+      // The tile's softmax.  `msk` is std::true_type / std::false_type for a copy
+      // specialised to masked / unmasked tiles, or a run-time bool for one copy that
+      // branches inside (only pass 1 masks: it sets hidden scores to -inf).
+      auto tile = [&](auto msk) -> bool {
+        tc_fence_after();
+        uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+        tmem_ld16x256_x16_wait(s_addr, sr);
+        if constexpr (kSepP) {
+          tc_fence_before();
+          mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+        }
 
-      // ---- pass 1: row maxima (log2 units) --------------------------------------
-      // ALiBi: the bias of column 8k + 2 t0 + c in row e is -slope |db[e] + 8k + c|,
-      // recomputed in both passes (cheaper than keeping the biased logits live).
-      // Under a causal mask a visible key is never after the query, so the bias
-      // is linear in the column there: slope (db[e] + 8k + c); hidden columns are
-      // set to -inf anyway.
-      float db[2], sdb[2];
+        // ---- pass 1: row maxima (log2 units) --------------------------------------
+        // ALiBi: the bias of column 8k + 2 t0 + c in row e is -slope |db[e] + 8k + c|,
+        // recomputed in both passes (cheaper than keeping the biased logits live).
+        // Under a causal mask a visible key is never after the query, so the bias
+        // is linear in the column there: slope (db[e] + 8k + c); hidden columns are
+        // set to -inf anyway.
+        float db[2], sdb[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        db[e] = static_cast<float>(n0 + 2 * t0 - pos[e]);
-        sdb[e] = slope_log2 * db[e];
-      }
-      auto bias = [&](int k, int c, int e) -> float {
-        if constexpr (kCausal) return fmaf(slope_log2, static_cast<float>(8 * k + c), sdb[e]);
-        return -slope_log2 * fabsf(db[e] + static_cast<float>(8 * k + c));
-      };
-      float mx[2] = {neg_inf(), neg_inf()};
-      if constexpr (ALIBI) {
-        auto biased = [&](auto msk) {
+        for (int e = 0; e < 2; ++e) {
+          db[e] = static_cast<float>(n0 + 2 * t0 - pos[e]);
+          sdb[e] = slope_log2 * db[e];
+        }
+        auto bias = [&](int k, int c, int e) -> float {
+          if constexpr (kCausal) return fmaf(slope_log2, static_cast<float>(8 * k + c), sdb[e]);
+          return -slope_log2 * fabsf(db[e] + static_cast<float>(8 * k + c));
+        };
+        float mx[2] = {neg_inf(), neg_inf()};
+        if constexpr (ALIBI) {
+          auto biased = [&](auto bmsk) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                  float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), scale_log2, bias(k, c, e));
+                  if constexpr (decltype(bmsk)::value) {
+                    if (hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
+                  }
+                  sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
+                  mx[e] = fmaxf(mx[e], y);
+                }
+          };
+          if (masked) biased(std::true_type{});
+          else biased(std::false_type{});
+        } else {
+          auto max_plain = [&] {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                mx[e] = max3(mx[e], __uint_as_float(sr[4 * k + 2 * e]),
+                             __uint_as_float(sr[4 * k + 2 * e + 1]));
+          };
+          // Hidden scores become -inf, so pass 2 needs no mask: 2^(-inf * scale - m)
+          // = 0 (scale_log2 > 0 here).
+          auto max_masked = [&] {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                  if (hidden(8 * k + 2 * t0 + c, e)) sr[4 * k + 2 * e + c] = __float_as_uint(neg_inf());
+                  mx[e] = fmaxf(mx[e], __uint_as_float(sr[4 * k + 2 * e + c]));
+                }
+          };
+          if (flag_on(msk)) max_masked();
+          else max_plain();
+        }
+        float alpha[2], nsub[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float pm = mx[e];
+          if constexpr (!ALIBI) pm *= scale_log2;
+          pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
+          pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
+          float m_use = m_ref[e];
+          if (pm > m_ref[e] + kTau) m_use = pm;  // also taken when m_ref is -inf
+          alpha[e] = (m_use == m_ref[e]) ? 1.f : ex2(m_ref[e] - m_use);
+          m_ref[e] = m_use;
+          nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
+        }
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
+
+        // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
+        // Hidden logits are -inf by now (pass 1), so one mask-free copy serves every tile.
+        f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
+        const f2 scale2 = {scale_log2, scale_log2};
+        auto pass2 = [&]() -> bool {
+          auto p_pair = [&](int k, int e) -> f2 {
+            const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
+            const f2 ns = {nsub[e], nsub[e]};
+            const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
+            const f2 p = {ex2(y.x), ex2(y.y)};
+            ps[e] = add2(ps[e], p);
+            return p;
+          };
+          if constexpr (kSepP) {
+            uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const f2 p = p_pair(k, e);
+                pk[2 * k + e] = pack2<BF16>(p.x, p.y);
+              }
+            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+            // P_t is still being read by P.V of the previous key tile.
+            if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
+              return false;
+            tc_fence_after();
+            tmem_st16x128_x16(p_addr, pk);
+          } else {
+            // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
+            // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
+            // lo pairs repetitions 4..7.
+#pragma unroll
+            for (int C = 0; C < 4; ++C) {
+              uint32_t pc[kSplitP ? 16 : 8];
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const f2 p = p_pair(4 * C + kk, e);
+                  const uint32_t hi = pack2<BF16>(p.x, p.y);
+                  pc[2 * kk + e] = hi;
+                  if constexpr (kSplitP) {
+                    const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
+                    const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
+                    pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
+                  }
+                }
+              if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
+              else tmem_st16x128_x4(p_addr + 32 * C, pc);
+            }
+            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+          }
+          return true;
+        };
+        if (!pass2()) return false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
+        // Rescale the output rows whose reference max moved (after the previous
+        // P.V has written O).
+        if (nc > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
+          if constexpr (!kSepP) {
+            if (!mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)) return false;
+            tc_fence_after();
+          }
+          uint32_t o[kOReg];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+          ld_o(o);
+#pragma unroll
+          for (int k = 0; k < D / 8; ++k)
 #pragma unroll
             for (int e = 0; e < 2; ++e)
 #pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), a.scale_log2, bias(k, c, e));
-                if constexpr (decltype(msk)::value) {
-                  if (hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
-                }
-                sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
-                mx[e] = fmaxf(mx[e], y);
-              }
-        };
-        if (masked) biased(std::true_type{});
-        else biased(std::false_type{});
-      } else if (!masked) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-            mx[e] = max3(mx[e], __uint_as_float(sr[4 * k + 2 * e]),
-                         __uint_as_float(sr[4 * k + 2 * e + 1]));
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              if (!hidden(8 * k + 2 * t0 + c, e))
-                mx[e] = fmaxf(mx[e], __uint_as_float(sr[4 * k + 2 * e + c]));
-      }
-      float alpha[2], nsub[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float pm = mx[e];
-        if constexpr (!ALIBI) pm = (pm == neg_inf()) ? pm : pm * a.scale_log2;
-        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
-        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
-        float m_use = m_ref[e];
-        if (pm > m_ref[e] + kTau) m_use = pm;  // also taken when m_ref is -inf
-        alpha[e] = (m_use == m_ref[e]) ? 1.f : ex2(m_ref[e] - m_use);
-        m_ref[e] = m_use;
-        nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
-      }
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
-
-      // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
-      // Instantiated separately for tiles with and without masking, so the
-      // per-element mask tests exist only in the masked copy (ALiBi's masked
-      // logits are already -inf, so its P needs none).
-      f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
-      const f2 scale2 = {a.scale_log2, a.scale_log2};
-      auto pass2 = [&](auto msk) -> bool {
-        constexpr bool kMsk = !ALIBI && decltype(msk)::value;
-        auto p_pair = [&](int k, int e) -> f2 {
-          const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
-          const f2 ns = {nsub[e], nsub[e]};
-          const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
-          f2 p = {ex2(y.x), ex2(y.y)};
-          if constexpr (kMsk) {
-            if (hidden(8 * k + 2 * t0, e)) p.x = 0.f;
-            if (hidden(8 * k + 2 * t0 + 1, e)) p.y = 0.f;
-          }
-          ps[e] = add2(ps[e], p);
-          return p;
-        };
-        if constexpr (kSepP) {
-          uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const f2 p = p_pair(k, e);
-              pk[2 * k + e] = pack2<BF16>(p.x, p.y);
-            }
-          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-          // P_t is still being read by P.V of the previous key tile.
-          if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
-            return false;
-          tc_fence_after();
-          tmem_st16x128_x16(p_addr, pk);
-        } else {
-          // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
-          // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
-          // lo pairs repetitions 4..7.
-#pragma unroll
-          for (int C = 0; C < 4; ++C) {
-            uint32_t pc[kSplitP ? 16 : 8];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const f2 p = p_pair(4 * C + kk, e);
-                const uint32_t hi = pack2<BF16>(p.x, p.y);
-                pc[2 * kk + e] = hi;
-                if constexpr (kSplitP) {
-                  const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
-                  const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
-                  pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
-                }
-              }
-            if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
-            else tmem_st16x128_x4(p_addr + 32 * C, pc);
-          }
-          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+              for (int c = 0; c < 2; ++c)
+                o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
+          st_o(o);
         }
         return true;
       };
-      if (!(ok = (!ALIBI && masked) ? pass2(std::true_type{}) : pass2(std::false_type{}))) break;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
-      // Rescale the output rows whose reference max moved (after the previous
-      // P.V has written O).
-      if (nc > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
-        if constexpr (!kSepP) {
-          if (!(ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))) break;
-          tc_fence_after();
-        }
-        uint32_t o[kOReg];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
-        ld_o(o);
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k)
-#pragma unroll
-          for (int e = 0; e < 2; ++e)
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-              o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
-        st_o(o);
-      }
+      // Two specialised copies where that compiles best (no register spills in the
+      // plain dense instances, measured); one copy elsewhere, and for ALiBi, whose
+      // biased-logit pass branches on `masked` itself.
+      if constexpr (kTileCopies) ok = masked ? tile(std::true_type{}) : tile(std::false_type{});
+      else ok = tile(!ALIBI && masked);
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[t]);

@@ -4,6 +4,7 @@
 // hang.  Everything here is a one-instruction wrapper; the kernels own the logic.
 #pragma once
 
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -421,6 +422,12 @@ __device__ __forceinline__ f2 add2(f2 a, f2 b) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
   return d;
 }
+
+// A mask flag given either at compile time (std::true_type / std::false_type,
+// for code specialised to one case) or at run time (bool).
+__device__ __forceinline__ constexpr bool flag_on(std::true_type) { return true; }
+__device__ __forceinline__ constexpr bool flag_on(std::false_type) { return false; }
+__device__ __forceinline__ bool flag_on(bool b) { return b; }
 
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {

@@ -142,6 +142,23 @@ def test_scale_zero_is_mean(mea):
                                                          dtype=torch.float64), atol=1e-3)
 
 
+@pytest.mark.parametrize("K,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_scale_zero_causal_is_running_mean(mea, K, dtype):
+    """Closed form under a causal mask (diagonal tiles masked): scale 0 -> row i
+    is the mean of v_0 .. v_i and lse_i = ln(i + 1)."""
+    g = torch.Generator().manual_seed(71)
+    M = 300
+    v = torch.randn(2, M, 2, K, generator=g).to(dtype)
+    q = torch.randn(2, M, 2, K, generator=g).to(dtype)
+    out, lse = mea.mea_fwd(q.to(DEV), v.to(DEV), v.to(DEV), bias="causal", scale=0.0)
+    torch.cuda.synchronize()
+    assert mea.read_device_status() == 0
+    cnt = torch.arange(1, M + 1, dtype=torch.float64)
+    ref = v.double().cumsum(1) / cnt.view(1, M, 1, 1)
+    assert_out_close(out, ref, "scale0_causal")
+    assert torch.allclose(lse.double().cpu(), torch.log(cnt).expand(2, 2, M), atol=1e-3)
+
+
 def test_repeatable(mea):
     """Two launches on the same input give bit-identical results."""
     p = synth.make_prefill("rep", 2, 300, 300, 4, 2, 128, "bf16", "causal", seed=80)
