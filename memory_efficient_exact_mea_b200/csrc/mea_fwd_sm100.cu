@@ -80,9 +80,28 @@ __device__ long long g_trace[kTraceCtas * kTraceSlots];
     if (blockIdx.x < kTraceCtas && (slot) < kTraceSlots)                           \
       g_trace[blockIdx.x * kTraceSlots + (slot)] = clock64();                      \
   } while (0)
+// Per-CTA globaltimer stamps (all CTAs up to kCtaTraceMax): slot 0 entry, 1 first
+// score tile of query tile 0 ready, 2 its key loop done, 3 its output stored,
+// 4 the SM the CTA ran on.
+constexpr int kCtaTraceMax = 4096;
+__device__ long long g_cta_trace[kCtaTraceMax * 8];
+#define MEA_CTA_AT(i)                                                              \
+  do {                                                                             \
+    if (blockIdx.x < kCtaTraceMax) {                                               \
+      long long t_;                                                                \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                       \
+      g_cta_trace[blockIdx.x * 8 + (i)] = t_;                                      \
+      unsigned sm_;                                                                \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(sm_));                             \
+      g_cta_trace[blockIdx.x * 8 + 4] = sm_;                                       \
+    }                                                                              \
+  } while (0)
 #else
 #define MEA_TRACE_AT(slot) \
   do {                     \
+  } while (0)
+#define MEA_CTA_AT(i) \
+  do {                \
   } while (0)
 #endif
 
@@ -140,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) MEA_CTA_AT(0);
 
   // ---- which (query block, head, batch or sequence) this CTA owns ----------
   // The query block varies fastest, so the blocks of one (head, batch) -- and
@@ -559,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
       if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
+      if (tracer && t == 0 && j == 0) MEA_CTA_AT(1);
       // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
       // need no masking for any row of the warp take the unmasked path.
       int n0 = j * kBN, kfirst = 0;
@@ -759,6 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++nc;
     }
     if constexpr (!SPARSE) nc = ntt;
+    if (tracer && t == 0) MEA_CTA_AT(2);
 
     // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
     if (ok && nc > 0) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
@@ -795,6 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (tracer && t == 0) MEA_CTA_AT(3);
   }
 
   tc_fence_before();
@@ -882,6 +905,11 @@ cudaError_t launch_fwd(const FwdLaunch& L, cudaStream_t stream) {
 extern "C" int mea_trace_read(long long* host, int n) {
   if (n > kTraceCtas * kTraceSlots) n = kTraceCtas * kTraceSlots;
   return cudaMemcpyFromSymbol(host, g_trace, n * sizeof(long long)) == cudaSuccess ? n : -1;
+}
+
+extern "C" int mea_trace_cta_read(long long* host, int n) {
+  if (n > kCtaTraceMax * 8) n = kCtaTraceMax * 8;
+  return cudaMemcpyFromSymbol(host, g_cta_trace, n * sizeof(long long)) == cudaSuccess ? n : -1;
 }
 #endif
 
