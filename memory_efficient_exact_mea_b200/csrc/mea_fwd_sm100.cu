@@ -50,22 +50,31 @@ constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceed
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D>
+// QB: Q buffers (two query tiles each); persistent instances double-buffer Q.
+template <int D, int QB>
 struct Smem {
   static constexpr int kChunks = D / 64;          // 64-element (128-byte) column chunks
   static constexpr int kChunkBytes = kBM * 128;   // one chunk of a 128-row tile
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kSlots = (D == 128) ? 4 : 8;
   static constexpr int kQ = 0;
-  static constexpr int kKV = 2 * kTileBytes;
+  static constexpr int kKV = QB * 2 * kTileBytes;
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1 + 2;
+  static constexpr int kNumBars = 2 * QB + 2 * kSlots + 2 + 2 + 2 + 1 + 2;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// A copy of x that the compiler cannot merge with other uses of x, so that x
+// need not stay live in a register until this point.
+__device__ __forceinline__ int opaque(int x) {
+  int y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 
 // Pipeline timeline for performance work: built only with -DMEA_TRACE, it
 // records clock64() at each pipeline event of the first kTraceCtas CTAs.
@@ -119,6 +128,13 @@ __device__ long long g_cta_trace[kCtaTraceMax * 8];
 // region is shifted back to end at the region's end (its first columns, seen by
 // an earlier tile or before row 0, are masked), so no row beyond a sequence's
 // valid rows is ever loaded.
+// Persistent instances: one CTA per SM walks the units blockIdx.x, + gridDim.x, ...
+// with every pipeline counter running on across units, so the next unit's Q, K/V
+// and first Q.K^T overlap the current unit's last steps and output epilogue.
+// Dense, unpacked, non-causal K = 64 fp16 without ALiBi (units of equal length).
+template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
+constexpr bool kPersistent = D == 64 && !BF16 && MASK == 0 && !ALIBI && MODE == kModeDense;
+
 template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -126,7 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmVn, const FwdArgs a) {
   constexpr bool SPARSE = (MODE == kModeSparse);
   constexpr bool kCache = (MODE == kModeCache);
-  using L = Smem<D>;
+  constexpr bool kPersist = kPersistent<D, BF16, MASK, ALIBI, MODE>;
+  constexpr int QB = kPersist ? 2 : 1;
+  using L = Smem<D, QB>;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
   constexpr bool kSplitP = BF16;  // P.V as (P_hi + P_lo).V for bf16
@@ -146,10 +164,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sKV = smem + L::kKV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + S;
-  uint64_t* s_full = bars + 1 + 2 * S;
+  uint64_t* q_full = bars;        // [QB]
+  uint64_t* q_empty = bars + QB;  // [QB] Q buffer free again (persistent instances)
+  uint64_t* kv_full = bars + 2 * QB;
+  uint64_t* kv_empty = bars + 2 * QB + S;
+  uint64_t* s_full = bars + 2 * QB + 2 * S;
   uint64_t* p_ready = s_full + 2;
   uint64_t* o_done = p_ready + 2;
   uint64_t* mma_done = o_done + 2;
@@ -167,10 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // from L2 instead of DRAM.  Under a causal mask the longest rows go first.
   int mb = blockIdx.x % a.num_mblocks;
   const int rem = blockIdx.x / a.num_mblocks;
-  const int h = rem % a.Hq;
-  const int unit = rem / a.Hq;
+  int h = rem % a.Hq;
+  int unit = rem / a.Hq;
   if (kCausal) mb = a.num_mblocks - 1 - mb;
-  const int kvh = h / a.group;
+  int kvh = h / a.group;
 
   int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, bidx = unit;
   if constexpr (kPacked) {
@@ -218,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *dst = *src;
     }
   }
-  const int m_base = mb * kFwdRowsPerCta;
+  int m_base = mb * kFwdRowsPerCta;
   if (m_base >= q_len) return;
   const int off = k_len - q_len;  // bottom-right causal alignment
 
@@ -241,7 +260,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       nt_tile[t] = mt < q_len ? n_past_tiles + (nn + kBN - 1) / kBN : 0;
     }
   }
-  const int nt = max(nt_tile[0], nt_tile[1]);
+  int nt = max(nt_tile[0], nt_tile[1]);
+
+  // Units this CTA runs: blockIdx.x, + gridDim.x, ... below n_units (persistent
+  // instances), or just its own.  next_unit() moves the per-unit values to unit
+  // cu (persistent instances only: dense, unpacked, non-causal).
+  const int n_units = kPersist ? a.num_mblocks * a.Hq * a.num_units : static_cast<int>(gridDim.x);
+  auto next_unit = [&](int cu) {
+    mb = cu % a.num_mblocks;
+    const int r = cu / a.num_mblocks;
+    h = r % a.Hq;
+    unit = r / a.Hq;
+    kvh = h / a.group;
+    bidx = unit;
+    m_base = mb * kFwdRowsPerCta;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) nt_tile[t] = m_base + t * kBM < q_len ? (k_len + kBN - 1) / kBN : 0;
+    nt = max(nt_tile[0], nt_tile[1]);
+  };
 
   // Key tile j: the row its copy starts at (in the cache or in the new rows),
   // the key position of its column 0 and its first column not already seen by
@@ -284,7 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- set-up -----------------------------------------------------------
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int qb = 0; qb < QB; ++qb) {
+      mbar_init(&q_full[qb], 1);
+      mbar_init(&q_empty[qb], 2);  // one commit per MMA-issuing thread (separate-P layout)
+    }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], kSepP ? 2 : 1);  // one release per MMA-issuing thread
@@ -319,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // ===================== TMA producer =====================================
-    if (lane == 0 && nt > 0) {
+    if (!kPersist && lane == 0 && nt > 0) {
       mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < L::kChunks; ++c)
@@ -348,6 +387,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = max(0, it - S); i < it; ++i)
         mbar_wait_drain(&kv_full[i % S], (i / S) & 1, a.status);
     }
+    // Persistent instances: Q double-buffered, ring and unit counters run on.
+    if (kPersist && lane == 0 && nt > 0) {
+      int it = 0, iu = 0;  // K/V ring copies and units, over all units
+      bool ok = true;
+      for (int cu = blockIdx.x;; cu += gridDim.x) {
+        if (iu > 0) next_unit(cu);
+        const int qb = iu % QB;
+        // The buffer's previous unit (QB units back) has finished its Q.K^T MMAs.
+        if (iu >= QB && !(ok = mbar_wait(&q_empty[qb], (iu / QB - 1) & 1, abort_flag, a.status)))
+          break;
+        mbar_arrive_expect_tx(&q_full[qb], 2 * L::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sQ + (2 * qb + t) * L::kTileBytes + c * L::kChunkBytes, &tmQ, &q_full[qb],
+                        c * 64, h, q0 + m_base + t * kBM, bidx);
+        for (int j = 0; j < nt; ++j) {
+          if constexpr (SPARSE) {
+            if (!uses(0, j) && !uses(1, j)) continue;
+          }
+          const KeyTile kt = key_tile(j);
+          for (int kv = 0; kv < 2; ++kv, ++it) {
+            const int slot = it % S;
+            if (!mbar_wait(&kv_empty[slot], ((it / S) & 1) ^ 1, abort_flag, a.status)) break;
+            mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
+            const CUtensorMap* map = kv ? &tmV : &tmK;
+            if (kCache && kt.fresh) map = kv ? &tmVn : &tmKn;
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
+                          c * 64, kvh, kt.row, bidx);
+          }
+          if (*abort_flag) break;
+        }
+        ++iu;
+        if (*abort_flag || cu + static_cast<int>(gridDim.x) >= n_units) break;
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      for (int i = max(0, iu - QB); i < iu; ++i)
+        mbar_wait_drain(&q_full[i % QB], (i / QB) & 1, a.status);
+      for (int i = max(0, it - S); i < it; ++i)
+        mbar_wait_drain(&kv_full[i % S], (i / S) & 1, a.status);
+    }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
     // ===================== MMA issuers, one per query tile ====================
     const int tile = warp - kMmaWarp;
@@ -358,9 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kv_addr = smem_u32(sKV);
       // S_t = Q_t K^T: both operands K-major; step k advances 16 elements (32 bytes)
       // inside a 128-byte swizzle row, then to the next 64-column chunk.
-      auto issue_qk = [&](int t, int slot) {
+      auto issue_qk = [&](int t, int slot, uint32_t q_buf) {
         const uint32_t d = tmem_base + t * kBN;
-        const uint32_t qa = q_addr + t * L::kTileBytes;
+        const uint32_t qa = q_buf + t * L::kTileBytes;
         const uint32_t kb = kv_addr + slot * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -400,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // li counts the key tiles in the ring (both query tiles), c the key tiles
       // this query tile has computed (its barrier phases).
       const int t = tile;
-      auto pv_step = [&](int lv, bool used, int cu) -> bool {
+      auto pv_step = [&](int lv, bool used, int cu, bool acc) -> bool {
         const int vs = (2 * lv + 1) % S;
         if (!mbar_wait(&kv_full[vs], ((2 * lv + 1) / S) & 1, abort_flag, a.status)) return false;
         MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 2);
@@ -408,14 +488,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&p_ready[t], cu & 1, abort_flag, a.status)) return false;
           MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 3);
           tc_fence_after();
-          issue_pv(t, vs, cu > 0);
+          issue_pv(t, vs, acc);
           umma_commit(&o_done[t]);
           MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 4);
         }
         umma_commit(&kv_empty[vs]);
         return true;
       };
-      if (kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
+      if (!kPersist && kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
         bool ok = true, prev_used = false;
         int li = 0, c = 0, prev_c = 0;
         for (int j = 0; j < nt && ok; ++j) {
@@ -434,19 +514,71 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = mbar_wait(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
               tc_fence_after();
             }
-            issue_qk(t, ks);
+            issue_qk(t, ks, q_addr);
             umma_commit(&s_full[t]);
             MEA_TRACE_AT(1024 + t * 256 + li * 8 + 1);
           }
           umma_commit(&kv_empty[ks]);
-          if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c);
+          if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c, prev_c > 0);
           prev_used = used;
           prev_c = c;
           c += used ? 1 : 0;
           ++li;
         }
         if constexpr (!SPARSE) li = nt;
-        if (ok && li > 0) pv_step(li - 1, prev_used, prev_c);
+        if (ok && li > 0) pv_step(li - 1, prev_used, prev_c, prev_c > 0);
+      }
+      // Over units the stream stays one step behind for P.V: the next unit's first
+      // Q.K^T goes out before this unit's last P.V.
+      if (kPersist && nt > 0) {
+        bool ok = true, prev_used = false, prev_acc = false;
+        // li: key tiles in the ring, c: key tiles this query tile computed (its
+        // barrier phases), both over all units; li0, c0: their values at the unit's start.
+        int li = 0, c = 0, prev_c = 0, li0 = 0, c0 = 0, iu = 0;
+        for (int cu = blockIdx.x;; cu += gridDim.x, ++iu) {
+          if (iu > 0) next_unit(cu);
+          const int qb = iu % QB;
+          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) break;
+          const uint32_t q_buf = q_addr + 2 * qb * L::kTileBytes;
+          for (int j = 0; j < nt && ok; ++j) {
+            const bool used = uses(t, j);
+            if constexpr (SPARSE) {
+              if (!used && !uses(1 - t, j)) continue;
+            } else {
+              li = li0 + j;  // dense: every key tile is in the ring and a tile uses a prefix
+              c = c0 + j;
+            }
+            const int ks = (2 * li) % S;
+            if (!(ok = mbar_wait(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + t * 256 + li * 8 + 0);
+            if (used) {
+              if (c > 0) {  // the softmax has read the previous S_t out of TMEM
+                if (!(ok = mbar_wait(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
+                tc_fence_after();
+              }
+              issue_qk(t, ks, q_buf);
+              umma_commit(&s_full[t]);
+              MEA_TRACE_AT(1024 + t * 256 + li * 8 + 1);
+            }
+            umma_commit(&kv_empty[ks]);
+            if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c, prev_acc);
+            prev_used = used;
+            prev_acc = c > c0;  // P.V accumulates after the unit's first key tile
+            prev_c = c;
+            c += used ? 1 : 0;
+            ++li;
+          }
+          if constexpr (!SPARSE) {
+            li = li0 + nt;
+            c = c0 + nt_tile[t];
+          }
+          li0 = li;
+          c0 = c;
+          // This unit's Q buffer is free once its Q.K^T MMAs have completed.
+          umma_commit(&q_empty[qb]);
+          if (!ok || cu + static_cast<int>(gridDim.x) >= n_units) break;
+        }
+        if (ok && li > 0) pv_step(li - 1, prev_used, prev_c, prev_acc);
       }
       // When P is written over S the chain softmax -> P.V -> Q.K^T of a tile is
       // serial, so one thread (warp 16) issues both tiles in the interleaved
@@ -471,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           MEA_TRACE_AT(1024 + li * 16 + 0);
           ++it;
           if (u0) {
-            issue_qk(0, kslot);
+            issue_qk(0, kslot, q_addr);
             MEA_TRACE_AT(1024 + li * 16 + 1);
             umma_commit(&s_full[0]);
           }
@@ -486,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(&kv_empty[vslot_prev]);
           }
           if (u1) {
-            issue_qk(1, kslot);
+            issue_qk(1, kslot, q_addr);
             MEA_TRACE_AT(1024 + li * 16 + 3);
             umma_commit(&s_full[1]);
           }
@@ -554,270 +686,281 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (D == 64) tmem_st16x256_x8(o_addr, o);
       else tmem_st16x256_x16(o_addr, o);
     };
-    const int ntt = nt_tile[t];
-    int rr[2], pos[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      rr[e] = m_base + t * kBM + lane0 + t1 + 8 * e;  // row inside the sequence
-      pos[e] = rr[e] + off;                           // its position in key coordinates
-    }
     const bool tracer = wt == 0 && lane == 0;
-    float slope_log2 = 0.f;
-    if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
     // A zero scale is taken as 1e-30 (the same softmax to fp32 precision for any
     // finite score), so that -inf * scale stays -inf for hidden keys.
     const float scale_log2 = fmaxf(a.scale_log2, 1e-30f);
-    float m_ref[2] = {neg_inf(), neg_inf()};  // reference max per row (log2 units)
-    float l_sum[2] = {0.f, 0.f};              // this thread's part of each row sum
     bool ok = true;
-    int nc = 0;
-    for (int j = 0; j < ntt; ++j) {
-      if constexpr (SPARSE) {
-        if (!uses(t, j)) continue;
-      } else {
-        nc = j;
-      }
-      if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
-      if (tracer && t == 0 && j == 0) MEA_CTA_AT(1);
-      // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
-      // need no masking for any row of the warp take the unmasked path.
-      int n0 = j * kBN, kfirst = 0;
-      if constexpr (kCache) {
-        const KeyTile kt = key_tile(j);
-        n0 = kt.pos;
-        kfirst = kt.lo;
-      }
-      int limit[2];
+    int nc = 0;  // key tiles this query tile has computed, over all units (barrier phases)
+    for (int cu = blockIdx.x;; cu += gridDim.x) {
+      if (kPersist) next_unit(cu);
+      const int nbase = nc;  // nc at the unit's start
+      const int ntt = nt_tile[t];
+      int rr[2], pos[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        limit[e] = k_len - n0;
-        if (kCausal) limit[e] = min(limit[e], pos[e] + 1 - n0);
+        rr[e] = m_base + t * kBM + lane0 + t1 + 8 * e;  // row inside the sequence
+        pos[e] = rr[e] + off;                           // its position in key coordinates
       }
-      const bool masked = __any_sync(0xffffffffu, limit[0] < kBN || limit[1] < kBN) ||
-                          (kCache && kfirst > 0);
-      auto hidden = [&](int col, int e) -> bool {
-        if constexpr (kCache) return col >= limit[e] || col < kfirst;
-        return col >= limit[e];
-      };
-      // The tile's softmax.  `msk` is std::true_type / std::false_type for a copy
-      // specialised to masked / unmasked tiles, or a run-time bool for one copy that
-      // branches inside (only pass 1 masks: it sets hidden scores to -inf).
-      auto tile = [&](auto msk) -> bool {
-        tc_fence_after();
-        uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
-        tmem_ld16x256_x16_wait(s_addr, sr);
-        if constexpr (kSepP) {
-          tc_fence_before();
-          mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
-        }
-
-        // ---- pass 1: row maxima (log2 units) --------------------------------------
-        // ALiBi: the bias of column 8k + 2 t0 + c in row e is -slope |db[e] + 8k + c|,
-        // recomputed in both passes (cheaper than keeping the biased logits live).
-        // Under a causal mask a visible key is never after the query, so the bias
-        // is linear in the column there: slope (db[e] + 8k + c); hidden columns are
-        // set to -inf anyway.
-        float db[2], sdb[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          db[e] = static_cast<float>(n0 + 2 * t0 - pos[e]);
-          sdb[e] = slope_log2 * db[e];
-        }
-        auto bias = [&](int k, int c, int e) -> float {
-          if constexpr (kCausal) return fmaf(slope_log2, static_cast<float>(8 * k + c), sdb[e]);
-          return -slope_log2 * fabsf(db[e] + static_cast<float>(8 * k + c));
-        };
-        float mx[2] = {neg_inf(), neg_inf()};
-        if constexpr (ALIBI) {
-          auto biased = [&](auto bmsk) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-#pragma unroll
-              for (int e = 0; e < 2; ++e)
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                  float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), scale_log2, bias(k, c, e));
-                  if constexpr (decltype(bmsk)::value) {
-                    if (hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
-                  }
-                  sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
-                  mx[e] = fmaxf(mx[e], y);
-                }
-          };
-          if (masked) biased(std::true_type{});
-          else biased(std::false_type{});
+      float slope_log2 = 0.f;
+      if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
+      float m_ref[2] = {neg_inf(), neg_inf()};  // reference max per row (log2 units)
+      float l_sum[2] = {0.f, 0.f};              // this thread's part of each row sum
+      for (int j = 0; j < ntt; ++j) {
+        if constexpr (SPARSE) {
+          if (!uses(t, j)) continue;
         } else {
-          auto max_plain = [&] {
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-#pragma unroll
-              for (int e = 0; e < 2; ++e)
-                mx[e] = max3(mx[e], __uint_as_float(sr[4 * k + 2 * e]),
-                             __uint_as_float(sr[4 * k + 2 * e + 1]));
-          };
-          // Hidden scores become -inf, so pass 2 needs no mask: 2^(-inf * scale - m)
-          // = 0 (scale_log2 > 0 here).
-          auto max_masked = [&] {
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-#pragma unroll
-              for (int e = 0; e < 2; ++e)
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                  if (hidden(8 * k + 2 * t0 + c, e)) sr[4 * k + 2 * e + c] = __float_as_uint(neg_inf());
-                  mx[e] = fmaxf(mx[e], __uint_as_float(sr[4 * k + 2 * e + c]));
-                }
-          };
-          if (flag_on(msk)) max_masked();
-          else max_plain();
+          nc = nbase + j;
         }
-        float alpha[2], nsub[2];
+        if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
+        if (tracer && t == 0 && j == 0 && cu == blockIdx.x) MEA_CTA_AT(1);
+        // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
+        // need no masking for any row of the warp take the unmasked path.
+        int n0 = j * kBN, kfirst = 0;
+        if constexpr (kCache) {
+          const KeyTile kt = key_tile(j);
+          n0 = kt.pos;
+          kfirst = kt.lo;
+        }
+        int limit[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          float pm = mx[e];
-          if constexpr (!ALIBI) pm *= scale_log2;
-          pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
-          pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
-          float m_use = m_ref[e];
-          if (pm > m_ref[e] + kTau) m_use = pm;  // also taken when m_ref is -inf
-          alpha[e] = (m_use == m_ref[e]) ? 1.f : ex2(m_ref[e] - m_use);
-          m_ref[e] = m_use;
-          nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
+          limit[e] = k_len - n0;
+          if (kCausal) limit[e] = min(limit[e], pos[e] + 1 - n0);
         }
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
-
-        // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
-        // Hidden logits are -inf by now (pass 1), so one mask-free copy serves every tile.
-        f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
-        const f2 scale2 = {scale_log2, scale_log2};
-        auto pass2 = [&]() -> bool {
-          auto p_pair = [&](int k, int e) -> f2 {
-            const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
-            const f2 ns = {nsub[e], nsub[e]};
-            const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
-            const f2 p = {ex2(y.x), ex2(y.y)};
-            ps[e] = add2(ps[e], p);
-            return p;
-          };
+        const bool masked = __any_sync(0xffffffffu, limit[0] < kBN || limit[1] < kBN) ||
+                            (kCache && kfirst > 0);
+        auto hidden = [&](int col, int e) -> bool {
+          if constexpr (kCache) return col >= limit[e] || col < kfirst;
+          return col >= limit[e];
+        };
+        // The tile's softmax.  `msk` is std::true_type / std::false_type for a copy
+        // specialised to masked / unmasked tiles, or a run-time bool for one copy that
+        // branches inside (only pass 1 masks: it sets hidden scores to -inf).
+        auto tile = [&](auto msk) -> bool {
+          tc_fence_after();
+          uint32_t sr[64];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+          tmem_ld16x256_x16_wait(s_addr, sr);
           if constexpr (kSepP) {
-            uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
+            tc_fence_before();
+            mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+          }
+
+          // ---- pass 1: row maxima (log2 units) --------------------------------------
+          // ALiBi: the bias of column 8k + 2 t0 + c in row e is -slope |db[e] + 8k + c|,
+          // recomputed in both passes (cheaper than keeping the biased logits live).
+          // Under a causal mask a visible key is never after the query, so the bias
+          // is linear in the column there: slope (db[e] + 8k + c); hidden columns are
+          // set to -inf anyway.
+          float db[2], sdb[2];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
+          for (int e = 0; e < 2; ++e) {
+            db[e] = static_cast<float>(n0 + 2 * t0 - pos[e]);
+            sdb[e] = slope_log2 * db[e];
+          }
+          auto bias = [&](int k, int c, int e) -> float {
+            if constexpr (kCausal) return fmaf(slope_log2, static_cast<float>(8 * k + c), sdb[e]);
+            return -slope_log2 * fabsf(db[e] + static_cast<float>(8 * k + c));
+          };
+          float mx[2] = {neg_inf(), neg_inf()};
+          if constexpr (ALIBI) {
+            auto biased = [&](auto bmsk) {
 #pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const f2 p = p_pair(k, e);
-                pk[2 * k + e] = pack2<BF16>(p.x, p.y);
-              }
-            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
-            // P_t is still being read by P.V of the previous key tile.
-            if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
-              return false;
-            tc_fence_after();
-            tmem_st16x128_x16(p_addr, pk);
+              for (int k = 0; k < 16; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                  for (int c = 0; c < 2; ++c) {
+                    float y = fmaf(__uint_as_float(sr[4 * k + 2 * e + c]), scale_log2, bias(k, c, e));
+                    if constexpr (decltype(bmsk)::value) {
+                      if (hidden(8 * k + 2 * t0 + c, e)) y = neg_inf();
+                    }
+                    sr[4 * k + 2 * e + c] = __float_as_uint(y);  // the biased logit, for pass 2
+                    mx[e] = fmaxf(mx[e], y);
+                  }
+            };
+            if (masked) biased(std::true_type{});
+            else biased(std::false_type{});
           } else {
-            // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
-            // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
-            // lo pairs repetitions 4..7.
+            auto max_plain = [&] {
 #pragma unroll
-            for (int C = 0; C < 4; ++C) {
-              uint32_t pc[kSplitP ? 16 : 8];
+              for (int k = 0; k < 16; ++k)
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
+                for (int e = 0; e < 2; ++e)
+                  mx[e] = max3(mx[e], __uint_as_float(sr[4 * k + 2 * e]),
+                               __uint_as_float(sr[4 * k + 2 * e + 1]));
+            };
+            // Hidden scores become -inf, so pass 2 needs no mask: 2^(-inf * scale - m)
+            // = 0 (scale_log2 > 0 here).
+            auto max_masked = [&] {
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                  for (int c = 0; c < 2; ++c) {
+                    if (hidden(8 * k + 2 * t0 + c, e)) sr[4 * k + 2 * e + c] = __float_as_uint(neg_inf());
+                    mx[e] = fmaxf(mx[e], __uint_as_float(sr[4 * k + 2 * e + c]));
+                  }
+            };
+            if (flag_on(msk)) max_masked();
+            else max_plain();
+          }
+          float alpha[2], nsub[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float pm = mx[e];
+            if constexpr (!ALIBI) pm *= scale_log2;
+            pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
+            pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
+            float m_use = m_ref[e];
+            if (pm > m_ref[e] + kTau) m_use = pm;  // also taken when m_ref is -inf
+            alpha[e] = (m_use == m_ref[e]) ? 1.f : ex2(m_ref[e] - m_use);
+            m_ref[e] = m_use;
+            nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
+          }
+          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
+
+          // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
+          // Hidden logits are -inf by now (pass 1), so one mask-free copy serves every tile.
+          f2 ps[2] = {{0.f, 0.f}, {0.f, 0.f}};
+          const f2 scale2 = {scale_log2, scale_log2};
+          auto pass2 = [&]() -> bool {
+            auto p_pair = [&](int k, int e) -> f2 {
+              const f2 v = {__uint_as_float(sr[4 * k + 2 * e]), __uint_as_float(sr[4 * k + 2 * e + 1])};
+              const f2 ns = {nsub[e], nsub[e]};
+              const f2 y = ALIBI ? add2(v, ns) : fma2(v, scale2, ns);  // ALiBi: v is the biased logit
+              const f2 p = {ex2(y.x), ex2(y.y)};
+              ps[e] = add2(ps[e], p);
+              return p;
+            };
+            if constexpr (kSepP) {
+              uint32_t pk[32];  // 16x128b order: register 2k + e = row e, keys 8k + 2 t0, +1
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                  const f2 p = p_pair(4 * C + kk, e);
-                  const uint32_t hi = pack2<BF16>(p.x, p.y);
-                  pc[2 * kk + e] = hi;
-                  if constexpr (kSplitP) {
-                    const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
-                    const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
-                    pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
-                  }
+                  const f2 p = p_pair(k, e);
+                  pk[2 * k + e] = pack2<BF16>(p.x, p.y);
                 }
-              if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
-              else tmem_st16x128_x4(p_addr + 32 * C, pc);
+              if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+              // P_t is still being read by P.V of the previous key tile.
+              if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
+                return false;
+              tc_fence_after();
+              tmem_st16x128_x16(p_addr, pk);
+            } else {
+              // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
+              // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
+              // lo pairs repetitions 4..7.
+#pragma unroll
+              for (int C = 0; C < 4; ++C) {
+                uint32_t pc[kSplitP ? 16 : 8];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const f2 p = p_pair(4 * C + kk, e);
+                    const uint32_t hi = pack2<BF16>(p.x, p.y);
+                    pc[2 * kk + e] = hi;
+                    if constexpr (kSplitP) {
+                      const f2 hf2 = {__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)};
+                      const f2 res = fma2(hf2, f2{-1.f, -1.f}, p);  // P - P_hi, exact in fp32
+                      pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
+                    }
+                  }
+                if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
+                else tmem_st16x128_x4(p_addr + 32 * C, pc);
+              }
+              if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
             }
-            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+            return true;
+          };
+          if (!pass2()) return false;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
+          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
+          // Rescale the output rows whose reference max moved (after the previous
+          // P.V has written O).
+          if (nc > nbase && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
+            if constexpr (!kSepP) {
+              if (!mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)) return false;
+              tc_fence_after();
+            }
+            uint32_t o[kOReg];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+            ld_o(o);
+#pragma unroll
+            for (int k = 0; k < D / 8; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                  o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
+            st_o(o);
           }
           return true;
         };
-        if (!pass2()) return false;
+        // Two specialised copies where that compiles best (no register spills in the
+        // plain dense instances, measured); one copy elsewhere, and for ALiBi, whose
+        // biased-logit pass branches on `masked` itself.
+        if constexpr (kTileCopies) ok = masked ? tile(std::true_type{}) : tile(std::false_type{});
+        else ok = tile(!ALIBI && masked);
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_ready[t]);
+        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
+        ++nc;
+      }
+      if constexpr (!SPARSE) nc = nbase + ntt;
+      if (tracer && t == 0 && cu == blockIdx.x) MEA_CTA_AT(2);
+
+      // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
+      // (Persistent instances recompute the rows here rather than keep them in
+      // registers through the key loop: that instance then compiles without spills.)
+      if constexpr (kPersist) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
-        // Rescale the output rows whose reference max moved (after the previous
-        // P.V has written O).
-        if (nc > 0 && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
-          if constexpr (!kSepP) {
-            if (!mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)) return false;
-            tc_fence_after();
-          }
-          uint32_t o[kOReg];  // register 4k + 2e + c: row e, column 8k + 2 t0 + c
+        for (int e = 0; e < 2; ++e) rr[e] = opaque(m_base + t * kBM + lane0 + t1 + 8 * e);
+      }
+      if (ok && nc > nbase) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
+      if (ok) {
+        tc_fence_after();
+        float l_tot[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          l_tot[e] = l_sum[e] + __shfl_xor_sync(0xffffffffu, l_sum[e], 1);
+          l_tot[e] += __shfl_xor_sync(0xffffffffu, l_tot[e], 2);
+        }
+        uint32_t o[kOReg];
+        if (nc > nbase) {
           ld_o(o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kOReg; ++i) o[i] = 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (rr[e] >= q_len) continue;
+          const float inv_l = l_tot[e] > 0.f ? 1.f / l_tot[e] : 0.f;
+          uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
+                          2 * (bidx * a.o_sb + static_cast<long long>(q0 + rr[e]) * a.o_sm +
+                               h * a.o_sh + 2 * t0);
 #pragma unroll
           for (int k = 0; k < D / 8; ++k)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-#pragma unroll
-              for (int c = 0; c < 2; ++c)
-                o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
-          st_o(o);
-        }
-        return true;
-      };
-      // Two specialised copies where that compiles best (no register spills in the
-      // plain dense instances, measured); one copy elsewhere, and for ALiBi, whose
-      // biased-logit pass branches on `masked` itself.
-      if constexpr (kTileCopies) ok = masked ? tile(std::true_type{}) : tile(std::false_type{});
-      else ok = tile(!ALIBI && masked);
-      if (!ok) break;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_ready[t]);
-      if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
-      ++nc;
-    }
-    if constexpr (!SPARSE) nc = ntt;
-    if (tracer && t == 0) MEA_CTA_AT(2);
-
-    // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
-    if (ok && nc > 0) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
-    if (ok) {
-      tc_fence_after();
-      float l_tot[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        l_tot[e] = l_sum[e] + __shfl_xor_sync(0xffffffffu, l_sum[e], 1);
-        l_tot[e] += __shfl_xor_sync(0xffffffffu, l_tot[e], 2);
-      }
-      uint32_t o[kOReg];
-      if (nc > 0) {
-        ld_o(o);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kOReg; ++i) o[i] = 0u;
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        if (rr[e] >= q_len) continue;
-        const float inv_l = l_tot[e] > 0.f ? 1.f / l_tot[e] : 0.f;
-        uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
-                        2 * (bidx * a.o_sb + static_cast<long long>(q0 + rr[e]) * a.o_sm +
-                             h * a.o_sh + 2 * t0);
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k)
-          *reinterpret_cast<uint32_t*>(orow + 16 * k) =
-              pack2<BF16>(__uint_as_float(o[4 * k + 2 * e]) * inv_l,
-                          __uint_as_float(o[4 * k + 2 * e + 1]) * inv_l);
-        if (t0 == 0 && a.lse != nullptr) {
-          const float lse = l_tot[e] > 0.f ? (m_ref[e] + __log2f(l_tot[e])) * kLn2 : neg_inf();
-          a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + rr[e]] = lse;
+            *reinterpret_cast<uint32_t*>(orow + 16 * k) =
+                pack2<BF16>(__uint_as_float(o[4 * k + 2 * e]) * inv_l,
+                            __uint_as_float(o[4 * k + 2 * e + 1]) * inv_l);
+          if (t0 == 0 && a.lse != nullptr) {
+            const float lse = l_tot[e] > 0.f ? (m_ref[e] + __log2f(l_tot[e])) * kLn2 : neg_inf();
+            a.lse[(static_cast<long long>(bidx) * a.Hq + h) * a.M + q0 + rr[e]] = lse;
+          }
         }
       }
+      if (tracer && t == 0 && cu == blockIdx.x) MEA_CTA_AT(3);
+      if (!kPersist || !ok || cu + static_cast<int>(gridDim.x) >= n_units) break;
     }
-    if (tracer && t == 0) MEA_CTA_AT(3);
   }
 
   tc_fence_before();
@@ -828,17 +971,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+cudaError_t sm_count(int* out) {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+    *out = cached[dev];
+    return cudaSuccess;
+  }
+  e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cached[dev] = *out;
+  return e;
+}
+
 template <int D, bool BF16, int MASK, bool ALIBI, int MODE = kModeDense>
 cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
   auto kern = fwd_kernel<D, BF16, MASK, ALIBI, MODE>;
-  const int smem = Smem<D>::kBytes;
+  constexpr bool kPersist = kPersistent<D, BF16, MASK, ALIBI, MODE>;
+  const int smem = Smem<D, kPersist ? 2 : 1>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(L.args.num_mblocks) * L.args.Hq *
                          L.args.num_units;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmKn,
+  long long ctas = grid;
+  if constexpr (kPersist) {
+    int sms = 0;
+    e = sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    ctas = min(grid, static_cast<long long>(sms));  // one CTA per SM
+  }
+  kern<<<static_cast<unsigned>(ctas), kThreads, smem, stream>>>(L.tmQ, L.tmK, L.tmV, L.tmKn,
                                                                   L.tmVn, L.args);
   return cudaGetLastError();
 }

@@ -125,6 +125,13 @@ def test_no_keys(mea):
     assert torch.all(torch.isneginf(lse))
 
 
+def test_many_units_per_cta(mea, orc):
+    """More 256-row query blocks than SMs, ragged rows and keys: CTAs that run
+    several blocks in turn (K=64 fp16 non-causal), every element checked."""
+    p = synth.make_prefill("units_b3_h24_m600_n520", 3, 600, 520, 24, 24, 64, "f16", "none", seed=72)
+    _check_full(mea, orc, p)
+
+
 def test_causal_more_queries_than_keys(mea, orc):
     """Causal with M > N: the first M - N rows see no key (out 0, lse -inf)."""
     p = synth.make_prefill("m_gt_n", 1, 300, 100, 2, 2, 64, "f16", "causal", seed=70)
