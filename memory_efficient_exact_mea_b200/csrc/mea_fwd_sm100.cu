@@ -26,8 +26,9 @@
 // from TMEM) | O0 | O1 (K columns each, the fp32 output accumulators).  At K = 64
 // with fp16, P has columns of its own instead (S0 | S1 | P0 | P1 | O0 | O1 =
 // 128 + 128 + 64 + 64 + 64 + 64), so each tile's next Q.K^T overlaps its softmax.
-// Shared memory: Q0, Q1 (loaded once) and a ring of key/value tiles, all in the
-// 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
+// Shared memory: Q0, Q1 (loaded once per unit; two such buffers in the persistent
+// instances, which walk several units per CTA) and a ring of key/value tiles, all
+// in the 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
 
 #include <type_traits>
