@@ -100,6 +100,9 @@ typedef enum {
  *         (a negative scale returns MEA_ERR_UNSUPPORTED: negate q instead).
  *
  * A query row that sees no key gets out = 0 and lse = -inf.
+ * Launch: one CTA per (256 query rows, query head, batch or sequence); for
+ * K = 64 fp16 without a mask or ALiBi one CTA per SM instead, each walking
+ * several such units in turn (same results, bit for bit run to run).
  * Returns MEA_OK or an error status; never synchronises.
  */
 int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse,

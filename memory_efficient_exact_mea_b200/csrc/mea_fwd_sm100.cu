@@ -31,6 +31,7 @@
 // in the 128-byte-swizzled layout the TMA writes and the MMA descriptors read.
 #include <math.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include "mea_internal.h"
@@ -974,16 +975,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Streaming multiprocessors of the current device (looked up once per device).
 cudaError_t sm_count(int* out) {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64];  // zero-initialised (static storage)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
-    *out = cached[dev];
-    return cudaSuccess;
+  if (dev >= 0 && dev < 64) {
+    const int n = cached[dev].load(std::memory_order_relaxed);
+    if (n > 0) {
+      *out = n;
+      return cudaSuccess;
+    }
   }
   e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) cached[dev] = *out;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cached[dev].store(*out, std::memory_order_relaxed);
   return e;
 }
 
