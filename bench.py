@@ -100,6 +100,22 @@ def decode_bytes(d: synth.Decode) -> float:
     return cache + 2.0 * d.B * d.Hq * d.K * el
 
 
+# Exponentials per clock per SM of the special-function unit (ex2.approx.f32),
+# measured on this B200 with a microbenchmark; clocks.max.sm of the part.
+EX2_PER_CLK_PER_SM = 16
+SM_MAX_MHZ = 1965.0
+
+
+def ex2_roofline(achieved_tflops: float, sms: int, K: int) -> dict:
+    """The prefill's second ceiling: one exponential per score, 4*K FLOP per score,
+    so the exponential unit alone allows sms * 16 * f_max * 4K FLOP/s."""
+    peak = sms * EX2_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6 * 4 * K / 1e12
+    return {"bound": "ex2 (special-function unit)", "achieved": round(achieved_tflops, 1),
+            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+            "peak_kind": f"derived: {sms} SMs x {EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
+                         f"{SM_MAX_MHZ:.0f} MHz x {4 * K} FLOP per score"}
+
+
 def load_peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
@@ -327,6 +343,7 @@ def run_ours(args, rank, world, local):
         "traffic_note": "mean DRAM read+write bytes per sweep launch (ncu, profiles/traffic.json);"
                         " algorithmic q+k+v+out = 65536*M bytes, mean 125.8 MB",
         "algorithmic": "4*K*H*B*M*N FLOP per launch",
+        "second_ceiling": ex2_roofline(achieved, torch.cuda.get_device_properties(dev).multi_processor_count, 64),
     }
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,

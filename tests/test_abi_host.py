@@ -223,3 +223,14 @@ def test_prefill_chunk_rejects_bad_arguments(lib):
     assert call(q=8) == UNSUPPORTED
     assert call(B=0) == 0
     assert call(M=0) == 0
+
+
+def test_bench_ex2_ceiling():
+    """The secondary roofline of the bench line: 148 SMs x 16 ex2/clk x 1965 MHz x
+    256 FLOP per score (K = 64) = 1191.2 TFLOP/s."""
+    import bench
+
+    r = bench.ex2_roofline(595.6, 148, 64)
+    assert r["peak"] == 1191.2
+    assert abs(r["frac"] - 0.5) < 1e-3  # 595.6 / 1191.2
+    assert r["unit"] == "TFLOP/s"
