@@ -497,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&kv_empty[vs]);
         return true;
       };
+      // Separate-P layout, one unit per CTA.
       if (!kPersist && kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
         bool ok = true, prev_used = false;
         int li = 0, c = 0, prev_c = 0;
@@ -530,8 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (!SPARSE) li = nt;
         if (ok && li > 0) pv_step(li - 1, prev_used, prev_c, prev_c > 0);
       }
-      // Over units the stream stays one step behind for P.V: the next unit's first
-      // Q.K^T goes out before this unit's last P.V.
+      // Persistent instances (separate-P layout, several units per CTA): the stream
+      // stays one step behind for P.V over unit boundaries too, so the next unit's
+      // first Q.K^T goes out before this unit's last P.V.
       if (kPersist && nt > 0) {
         bool ok = true, prev_used = false, prev_acc = false;
         // li: key tiles in the ring, c: key tiles this query tile computed (its
