@@ -20,12 +20,14 @@ import os
 
 import torch
 
-__all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_prefill_chunk", "mea_bwd", "mea_decode", "mea_decode_workspace_size", "mea_decode_chunk",
-           "read_device_status", "status_string", "MeaError", "BIAS", "LIB_PATH", "lib"]
+__all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_prefill_chunk", "mea_bwd", "mea_decode",
+           "mea_decode_workspace_size", "mea_decode_chunk", "read_device_status", "status_string",
+           "MeaError", "BIAS", "BWD_PREP", "BWD_MAIN", "BWD_DQ", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
 
 BIAS = {"none": 0, "causal": 1, "blockdiag": 2, "blockdiag_causal": 3}
+BWD_PREP, BWD_MAIN, BWD_DQ = 1, 2, 4  # stages of the backward (mea_bwd_stages)
 _DTYPE = {torch.float16: 0, torch.bfloat16: 1}
 _i64x3 = ctypes.c_int64 * 3
 
@@ -41,7 +43,7 @@ class MeaError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m memory_efficient_exact_mea_b200.build`")
+            f"{LIB_PATH} is not built; run `python memory_efficient_exact_mea_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.mea_fwd.restype = i
@@ -62,6 +64,8 @@ def _load() -> ctypes.CDLL:
     L.mea_bwd_workspace_size.argtypes = [i, i, i, i]
     L.mea_bwd.restype = i
     L.mea_bwd.argtypes = [vp] * 9 + [i] * 8 + [vp, vp, i, i, i, i, f, vp, sz, vp]
+    L.mea_bwd_stages.restype = i
+    L.mea_bwd_stages.argtypes = [vp] * 9 + [i] * 8 + [vp, vp, i, i, i, i, f, vp, sz, i, vp]
     L.mea_decode_chunk.restype = i
     L.mea_decode_chunk.argtypes = []
     L.mea_status_string.restype = ctypes.c_char_p
@@ -84,9 +88,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device=None):
+    """The CUDA stream handle to launch on: `stream`, else the current stream of
+    `device` (a torch.device, default the current device)."""
+    if stream is None:
+        if _raw_stream is not None and device is not None and device.index is not None:
+            return ctypes.c_void_p(_raw_stream(device.index))
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _check(fn, rc):
@@ -94,12 +106,46 @@ def _check(fn, rc):
         raise MeaError(fn, rc)
 
 
+_STRIDES: dict = {}  # (sb, sm, sh) -> ctypes int64[3], reused across calls (read-only)
+
+
 def _bmhk_strides(t: torch.Tensor, name: str):
-    if t.dim() != 4:
+    st = t.stride()
+    if len(st) != 4:
         raise ValueError(f"{name} must be [B, rows, heads, K]")
-    if t.stride(3) != 1:
+    if st[3] != 1:
         raise ValueError(f"{name}: the last dimension must be contiguous")
-    return _i64x3(t.stride(0), t.stride(1), t.stride(2))
+    key = st[:3]
+    arr = _STRIDES.get(key)
+    if arr is None:
+        if len(_STRIDES) > 4096:
+            _STRIDES.clear()
+        arr = _STRIDES[key] = _i64x3(*key)
+    return arr
+
+
+def _grouped_views(q, k, v, out):
+    """The 5-D grouped-query layout as 4-D views (no copy): q [B,M,G,H,K] ->
+    [B,M,G*H,K] (query head g*H + r); k, v [B,N,G,1,K], or [B,N,G,H,K] expanded
+    along H with stride 0, -> [B,N,G,K] (key/value head g, shared by the H query
+    heads of group g); k, v with a real H axis -> [B,N,G*H,K]."""
+    B, M, G, H, K = q.shape
+    if k.dim() != 5 or v.dim() != 5 or k.shape[:3] != v.shape[:3] or k.shape[2] != G:
+        raise ValueError("5-D q [B,M,G,H,K] needs k, v [B,N,G,1|H,K]")
+
+    def flat(t, name):
+        if t.shape[3] != 1 and t.stride(2) != t.shape[3] * t.stride(3):
+            raise ValueError(f"{name}: the group and head axes must merge into one (a view)")
+        return t.flatten(2, 3)
+
+    def kv4(t, name):
+        if t.shape[3] == 1 or t.stride(3) == 0:
+            return t[:, :, :, 0]
+        return flat(t, name)
+
+    q4 = flat(q, "q")
+    o4 = None if out is None else flat(out, "out")
+    return q4, kv4(k, "k"), kv4(v, "v"), o4
 
 
 def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool = False,
@@ -113,7 +159,18 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
     kinds take B == 1 and int32 CUDA offsets ``seqstart_q`` (and ``seqstart_k``);
     ``max_seqlen_q`` is the longest query sequence (read from the offsets, with a
     device-to-host copy, when not given).
+
+    Grouped-query 5-D layout: q [B,M,G,H,K] with k, v [B,N,G,1,K] (or expanded to
+    [B,N,G,H,K] with stride 0) is the same call with Hq = G*H query heads and
+    Hkv = G key/value heads, query head g*H + r reading key/value head g; out is
+    returned as [B,M,G,H,K] and lse as [B,G*H,M].
     """
+    if q.dim() == 5:
+        shape5 = tuple(q.shape)
+        q, k, v, out4 = _grouped_views(q, k, v, out)
+        o, l = mea_fwd(q, k, v, bias, scale, alibi, seqstart_q, seqstart_k, max_seqlen_q,
+                       max_seqlen_k, out4, lse, return_lse, stream)
+        return o.view(shape5) if out is None else out, l
     B, M, Hq, K = q.shape
     N, Hkv = k.shape[1], k.shape[2]
     if q.dtype not in _DTYPE or k.dtype != q.dtype or v.dtype != q.dtype:
@@ -148,7 +205,7 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
                      _bmhk_strides(q, "q"), _bmhk_strides(k, "k"), _bmhk_strides(v, "v"),
                      _bmhk_strides(out, "out"), _DTYPE[q.dtype], kind, _ptr(seqstart_q),
                      _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k), int(bool(alibi)),
-                     scale, _stream(stream))
+                     scale, _stream(stream, q.device))
     _check("mea_fwd", rc)
     return out, lse
 
@@ -187,7 +244,7 @@ def mea_fwd_block_sparse(q, k, v, block_mask, bias: str = "none", scale: float |
                                   Hkv, K, _bmhk_strides(q, "q"), _bmhk_strides(k, "k"),
                                   _bmhk_strides(v, "v"), _bmhk_strides(out, "out"),
                                   _DTYPE[q.dtype], BIAS[bias], _ptr(block_mask), mst,
-                                  int(bool(alibi)), scale, _stream(stream))
+                                  int(bool(alibi)), scale, _stream(stream, q.device))
     _check("mea_fwd_block_sparse", rc)
     return out, lse
 
@@ -228,7 +285,7 @@ def mea_prefill_chunk(q, k_new, v_new, k_cache, v_cache, cache_seqlens, q_seqlen
                                _bmhk_strides(k_cache, "k_cache"),
                                _bmhk_strides(v_cache, "v_cache"), _bmhk_strides(out, "out"),
                                _DTYPE[q.dtype], int(bool(causal)), int(bool(alibi)), scale,
-                               _stream(stream))
+                               _stream(stream, q.device))
     _check("mea_prefill_chunk", rc)
     return out, lse
 
@@ -236,9 +293,13 @@ def mea_prefill_chunk(q, k_new, v_new, k_cache, v_cache, cache_seqlens, q_seqlen
 def mea_bwd(q, k, v, out, dout, lse, bias: str = "none", scale: float | None = None,
             alibi: bool = False, seqstart_q=None, seqstart_k=None,
             max_seqlen_q: int | None = None, max_seqlen_k: int | None = None,
-            dq=None, dk=None, dv=None, workspace=None, stream=None):
+            dq=None, dk=None, dv=None, workspace=None, stages: int = 7, stream=None):
     """Attention backward.  Contiguous q/out/dout [B,M,Hq,K], k/v [B,N,Hkv,K] and the
-    forward's lse [B,Hq,M] -> (dq, dk, dv) shaped like q, k, v."""
+    forward's lse [B,Hq,M] -> (dq, dk, dv) shaped like q, k, v.
+
+    ``stages`` (bitwise OR of BWD_PREP, BWD_MAIN, BWD_DQ; default all) runs only
+    those launches of the backward (mea_bwd_stages); running them one at a time
+    with the same arguments and workspace equals one full call."""
     B, M, Hq, K = q.shape
     N, Hkv = k.shape[1], k.shape[2]
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
@@ -266,10 +327,11 @@ def mea_bwd(q, k, v, out, dout, lse, bias: str = "none", scale: float | None = N
     else:
         seqstart_q = seqstart_k = None
         max_seqlen_q = max_seqlen_k = 0
-    rc = lib.mea_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq),
-                     _ptr(dk), _ptr(dv), B, M, N, Hq, Hkv, K, _DTYPE[q.dtype], kind,
-                     _ptr(seqstart_q), _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k),
-                     int(bool(alibi)), scale, _ptr(workspace), ws_bytes, _stream(stream))
+    rc = lib.mea_bwd_stages(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                            _ptr(dq), _ptr(dk), _ptr(dv), B, M, N, Hq, Hkv, K, _DTYPE[q.dtype],
+                            kind, _ptr(seqstart_q), _ptr(seqstart_k), ns, int(max_seqlen_q),
+                            int(max_seqlen_k), int(bool(alibi)), scale, _ptr(workspace), ws_bytes,
+                            int(stages), _stream(stream, q.device))
     _check("mea_bwd", rc)
     return dq, dk, dv
 
@@ -311,7 +373,7 @@ def mea_decode(q, k_cache, v_cache, kv_seqstart, max_kv_len: int, scale: float |
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = lib.mea_decode(_ptr(q3), _ptr(k_cache), _ptr(v_cache), _ptr(kv_seqstart), _ptr(out),
                         _ptr(lse), B, Hq, Hkv, K, T, int(max_kv_len), _DTYPE[q.dtype],
-                        int(bool(alibi)), scale, _ptr(workspace), ws_bytes, _stream(stream))
+                        int(bool(alibi)), scale, _ptr(workspace), ws_bytes, _stream(stream, q.device))
     _check("mea_decode", rc)
     return out, lse
 

@@ -262,3 +262,90 @@ def chunk_prefill() -> Chunk:
     past = lengths(8, 1024, 8192, generator(1008)).tolist()
     return make_chunk("chunk512_b8_past1k-8k_hq32_hkv8_k128_bf16", past, 512, 8704, 32, 8, 128,
                       "bf16", True, seed=1009)
+
+
+# ---------------------------------------------------------------------------
+# Shaped inputs: score ranges that move across key tiles.  Row maxima of the
+# plain N(0,1) draws change little from one key tile to the next; these make
+# them climb (or fall) by large factors along the key axis, or put scores in
+# the hundreds, or place tile-to-tile jumps of chosen size.
+# ---------------------------------------------------------------------------
+def ramp(n: int, lo: float, hi: float) -> torch.Tensor:
+    """n factors going linearly from lo to hi (float32; lo alone when n == 1)."""
+    if n <= 1:
+        return torch.full((max(n, 0),), float(lo), dtype=torch.float32)
+    return torch.linspace(float(lo), float(hi), n, dtype=torch.float32)
+
+
+def scale_rows(x: torch.Tensor, factors: torch.Tensor, dim: int = 1) -> torch.Tensor:
+    """x with slice i along `dim` multiplied by factors[i] (float32 product, cast
+    back to x's dtype)."""
+    shape = [1] * x.dim()
+    shape[dim] = -1
+    return (x.to(torch.float32) * factors.view(shape)).to(x.dtype)
+
+
+def ramp_keys(p: Prefill, lo: float, hi: float) -> Prefill:
+    """Keys of every sequence multiplied by factors going from lo to hi along the
+    sequence's key positions (per packed segment when the batch is packed)."""
+    if p.seq_lens_q is None:
+        f = ramp(p.N, lo, hi)
+    else:
+        lens = p.seq_lens_k if p.seq_lens_k is not None else p.seq_lens_q
+        f = torch.cat([ramp(int(n), lo, hi) for n in lens]) if len(lens) else ramp(0, lo, lo)
+    p.k = scale_rows(p.k, f, 1)
+    p.name += f"_keys{lo:g}to{hi:g}"
+    return p
+
+
+def amplify(p: Prefill, c: float) -> Prefill:
+    """q and k multiplied by c (scores grow by c^2)."""
+    p.q = (p.q.to(torch.float32) * c).to(p.q.dtype)
+    p.k = (p.k.to(torch.float32) * c).to(p.k.dtype)
+    p.name += f"_x{c:g}"
+    return p
+
+
+def ramp_chunk_keys(c: Chunk, lo: float, hi: float) -> Chunk:
+    """Cached and new keys multiplied by factors from lo to hi along each
+    sequence's key positions 0 .. past + q_len - 1 (the new rows continue the
+    cached ones)."""
+    for b, (past, n) in enumerate(zip(c.past, c.q_lens)):
+        f = ramp(past + n, lo, hi)
+        if past:
+            c.k_cache[b, :past] = scale_rows(c.k_cache[b, :past], f[:past], 0)
+        if n:
+            c.k_new[b, :n] = scale_rows(c.k_new[b, :n], f[past:], 0)
+    c.name += f"_keys{lo:g}to{hi:g}"
+    return c
+
+
+def tile_step_scores(name: str, B: int, N: int, Hq: int, K: int, dtype: str, steps, tile: int,
+                     seed: int, bias: str = "none", noise: float = 0.0) -> Prefill:
+    """Scores that are constant within each block of `tile` keys and move by the
+    given amounts from block to block: q = e_0 (plus `noise` N(0,1) on the other
+    components), key j has component 0 equal to the running sum of steps[:j // tile]
+    and N(0,1) elsewhere, so row i's score with key j is exactly that sum (times
+    the scale) when noise = 0.  Batch b uses the steps rotated by b.  Values are
+    exact in fp16/bf16 when the steps are multiples of 1/16 below 64.  M = N, Hkv = Hq."""
+    g = generator(seed)
+    p = Prefill(name, B, N, N, Hq, Hq, K, dtype, bias, False, seed)
+    q = torch.zeros((B, N, Hq, K), dtype=torch.float32)
+    q[..., 0] = 1.0
+    if noise:
+        q[..., 1:] = noise * torch.randn((B, N, Hq, K - 1), generator=g, dtype=torch.float32)
+    k = torch.randn((B, N, Hq, K), generator=g, dtype=torch.float32)
+    steps = [float(s) for s in steps]
+    nblk = -(-N // tile)
+    for b in range(B):
+        rot = steps[b % len(steps):] + steps[:b % len(steps)]
+        level, levels = 0.0, []
+        for t in range(nblk):
+            levels.append(level)
+            level += rot[t % len(rot)]
+        col = torch.tensor(levels, dtype=torch.float32).repeat_interleave(tile)[:N]
+        k[b, :, :, 0] = col.view(N, 1)
+    p.q = q.to(DTYPES[dtype])
+    p.k = k.to(DTYPES[dtype])
+    p.v = randn((B, N, Hq, K), dtype, g)
+    return p

@@ -151,6 +151,17 @@ def _bwd(lib, **kw):
                        ctypes.c_float(a["scale"]), vp(a["ws"]), a["wsb"], vp(a["stream"]))
 
 
+def test_bwd_stages_rejects_bad_masks(lib):
+    """mea_bwd_stages takes a nonzero OR of its three stage bits."""
+    INVALID = -1
+    vp = ctypes.c_void_p
+    for stages in (0, 8, -1):
+        rc = lib.mea_bwd_stages(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(16),
+                                vp(16), 2, 100, 100, 8, 2, 128, 1, 1, None, None, 0, 0, 0, 0,
+                                ctypes.c_float(0.1), vp(256), 1 << 30, stages, None)
+        assert rc == INVALID, stages
+
+
 def test_bwd_workspace_size():
     import memory_efficient_exact_mea_b200 as m
 
@@ -226,11 +237,15 @@ def test_prefill_chunk_rejects_bad_arguments(lib):
 
 
 def test_bench_ex2_ceiling():
-    """The secondary roofline of the bench line: 148 SMs x 16 ex2/clk x 1965 MHz x
-    256 FLOP per score (K = 64) = 1191.2 TFLOP/s."""
+    """The secondary roofline of the bench line: 148 SMs x 16 ex2/clk x the SM
+    clock x 256 FLOP per score (K = 64): 1191.2 TFLOP/s at the 1965 MHz maximum,
+    1122.7 at a sampled 1852 MHz."""
     import bench
 
     r = bench.ex2_roofline(595.6, 148, 64)
     assert r["peak"] == 1191.2
     assert abs(r["frac"] - 0.5) < 1e-3  # 595.6 / 1191.2
     assert r["unit"] == "TFLOP/s"
+    r = bench.ex2_roofline(561.35, 148, 64, sm_mhz=1852.0)
+    assert r["peak"] == 1122.7
+    assert abs(r["frac"] - 0.5) < 1e-3

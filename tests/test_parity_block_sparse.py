@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import BIAS_CODE, assert_lse_close, assert_out_close
+from parity_util import BIAS_CODE, Guarded, assert_lse_close, assert_out_close
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -28,10 +28,16 @@ def orc():
 
 
 def _run(mea, p, mask):
+    """One mea_fwd_block_sparse with out and lse between guard bands."""
+    go = Guarded((p.B, p.M, p.Hq, p.K), p.q.dtype, DEV, fill=float("nan"))
+    gl = Guarded((p.B, p.Hq, p.M), torch.float32, DEV, fill=float("nan"))
     out, lse = mea.mea_fwd_block_sparse(p.q.to(DEV), p.k.to(DEV), p.v.to(DEV), mask.to(DEV),
-                                        bias=p.bias, scale=p.scale, alibi=p.alibi)
+                                        bias=p.bias, scale=p.scale, alibi=p.alibi, out=go.t,
+                                        lse=gl.t)
     torch.cuda.synchronize()
     assert mea.read_device_status() == 0
+    go.check(p.name + " out")
+    gl.check(p.name + " lse")
     return out, lse
 
 

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import assert_lse_close, assert_out_close
+from parity_util import Guarded, assert_lse_close, assert_out_close
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -31,12 +31,15 @@ def _run(mea, c: synth.Chunk, kc=None, vc=None):
     vc = c.v_cache.to(DEV) if vc is None else vc
     cl = torch.tensor(c.past, dtype=torch.int32, device=DEV)
     ql = torch.tensor(c.q_lens, dtype=torch.int32, device=DEV)
-    out = torch.zeros((c.B, c.M, c.Hq, c.K), dtype=c.q.dtype, device=DEV)
-    lse = torch.full((c.B, c.Hq, c.M), 123.0, device=DEV)
+    go = Guarded((c.B, c.M, c.Hq, c.K), c.q.dtype, DEV, fill=0.0)
+    gl = Guarded((c.B, c.Hq, c.M), torch.float32, DEV, fill=123.0)
+    out, lse = go.t, gl.t
     mea.mea_prefill_chunk(c.q.to(DEV), c.k_new.to(DEV), c.v_new.to(DEV), kc, vc, cl, ql,
                           causal=c.causal, scale=c.scale, alibi=c.alibi, out=out, lse=lse)
     torch.cuda.synchronize()
     assert mea.read_device_status() == 0
+    go.check(c.name + " out")
+    gl.check(c.name + " lse")
     return out, lse, kc, vc
 
 

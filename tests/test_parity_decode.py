@@ -6,7 +6,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import assert_lse_close, assert_out_close
+from parity_util import Guarded, assert_lse_close, assert_out_close
 
 pytestmark = pytest.mark.gpu
 
@@ -26,12 +26,20 @@ def orc():
 
 
 def _run(mea, d: synth.Decode, max_kv_len=None):
+    """One mea_decode with out, lse and the workspace between guard bands."""
     st = d.kv_seqstart.to(DEV)
-    out, lse = mea.mea_decode(d.q.to(DEV), d.k_cache.to(DEV), d.v_cache.to(DEV), st,
-                              d.max_kv_len if max_kv_len is None else max_kv_len,
-                              scale=d.scale, alibi=d.alibi)
+    mkl = d.max_kv_len if max_kv_len is None else max_kv_len
+    go = Guarded((d.B, 1, d.Hq, d.K), d.q.dtype, DEV, fill=float("nan"))
+    gl = Guarded((d.B, d.Hq), torch.float32, DEV, fill=float("nan"))
+    gw = Guarded((max(1, mea.mea_decode_workspace_size(d.B, d.Hq, d.Hkv, d.K, mkl)),),
+                 torch.uint8, DEV)
+    out, lse = mea.mea_decode(d.q.to(DEV), d.k_cache.to(DEV), d.v_cache.to(DEV), st, mkl,
+                              scale=d.scale, alibi=d.alibi, out=go.t, lse=gl.t, workspace=gw.t)
     torch.cuda.synchronize()
     assert mea.read_device_status() == 0
+    go.check(d.name + " out")
+    gl.check(d.name + " lse")
+    gw.check(d.name + " workspace")
     return out, lse
 
 

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import BIAS_CODE, assert_lse_close, assert_out_close
+from parity_util import BIAS_CODE, Guarded, assert_lse_close, assert_out_close
 
 pytestmark = pytest.mark.gpu
 
@@ -27,13 +27,19 @@ def orc():
 
 
 def _run_gpu(mea, p: synth.Prefill):
+    """One mea_fwd with out and lse between guard bands (checked untouched)."""
     q, k, v = p.q.to(DEV), p.k.to(DEV), p.v.to(DEV)
     kw = {}
     if p.bias.startswith("blockdiag"):
         kw = dict(seqstart_q=p.seqstart_q.to(DEV), seqstart_k=p.seqstart_k.to(DEV))
-    out, lse = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, **kw)
+    go = Guarded((p.B, p.M, p.Hq, p.K), q.dtype, DEV, fill=float("nan"))
+    gl = Guarded((p.B, p.Hq, p.M), torch.float32, DEV, fill=float("nan"))
+    out, lse = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, out=go.t,
+                           lse=gl.t, **kw)
     torch.cuda.synchronize()
     assert mea.read_device_status() == 0
+    go.check(p.name + " out")
+    gl.check(p.name + " lse")
     return out, lse
 
 
@@ -230,3 +236,29 @@ def test_repeatable_each_layout(mea, K, dtype, bias):
     for _ in range(5):
         again = _run_gpu(mea, p)
         assert torch.equal(again[0], first[0]) and torch.equal(again[1], first[1])
+
+
+@pytest.mark.parametrize("expanded", [False, True])
+def test_grouped_5d_layout(mea, orc, expanded):
+    """The 5-D grouped-query layout of the xFormers tutorial ("Dimotrazione di
+    Gruppo Query Attention (GQA)"): q [B,M,G,H,K] with k, v [B,N,G,1,K] (or expanded
+    along H with stride 0).  Query head (g, r) must attend with key/value head g:
+    compared with the oracle on the same problem with the key/value heads
+    repeated explicitly (every query head its own copy)."""
+    B, M, N, G, H, K = 2, 300, 260, 2, 4, 128
+    g = synth.generator(90)
+    q5 = synth.randn((B, M, G, H, K), "bf16", g)
+    k5 = synth.randn((B, N, G, 1, K), "bf16", g)
+    v5 = synth.randn((B, N, G, 1, K), "bf16", g)
+    kd, vd = k5.to(DEV), v5.to(DEV)
+    if expanded:
+        kd, vd = kd.expand(B, N, G, H, K), vd.expand(B, N, G, H, K)
+    out, lse = mea.mea_fwd(q5.to(DEV), kd, vd, bias="causal", scale=K ** -0.5)
+    torch.cuda.synchronize()
+    assert mea.read_device_status() == 0
+    assert tuple(out.shape) == (B, M, G, H, K) and tuple(lse.shape) == (B, G * H, M)
+    k_rep = k5.expand(B, N, G, H, K).reshape(B, N, G * H, K)
+    v_rep = v5.expand(B, N, G, H, K).reshape(B, N, G * H, K)
+    ro, rl = orc.attention(q5.reshape(B, M, G * H, K), k_rep, v_rep, bias=1, scale=K ** -0.5)
+    assert_out_close(out.reshape(B, M, G * H, K), ro, "5-D grouped")
+    assert_lse_close(lse, rl, "5-D grouped")
