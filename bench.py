@@ -106,14 +106,17 @@ EX2_PER_CLK_PER_SM = 16
 SM_MAX_MHZ = 1965.0
 
 
-def ex2_roofline(achieved_tflops: float, sms: int, K: int) -> dict:
+def ex2_roofline(achieved_tflops: float, sms: int, K: int, sm_mhz: float | None = None) -> dict:
     """The prefill's second ceiling: one exponential per score, 4*K FLOP per score,
-    so the exponential unit alone allows sms * 16 * f_max * 4K FLOP/s."""
-    peak = sms * EX2_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6 * 4 * K / 1e12
+    so the exponential unit alone allows sms * 16 * f * 4K FLOP/s at SM clock f
+    (the median sampled during the timed region when known, else the maximum)."""
+    f = SM_MAX_MHZ if not sm_mhz else float(sm_mhz)
+    peak = sms * EX2_PER_CLK_PER_SM * f * 1e6 * 4 * K / 1e12
     return {"bound": "ex2 (special-function unit)", "achieved": round(achieved_tflops, 1),
             "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
             "peak_kind": f"derived: {sms} SMs x {EX2_PER_CLK_PER_SM} ex2/clk/SM (measured) x "
-                         f"{SM_MAX_MHZ:.0f} MHz x {4 * K} FLOP per score"}
+                         f"{f:.0f} MHz ({'sampled median' if sm_mhz else 'maximum'} SM clock) x "
+                         f"{4 * K} FLOP per score"}
 
 
 def load_peaks():
@@ -343,7 +346,9 @@ def run_ours(args, rank, world, local):
         "traffic_note": "mean DRAM read+write bytes per sweep launch (ncu, profiles/traffic.json);"
                         " algorithmic q+k+v+out = 65536*M bytes, mean 125.8 MB",
         "algorithmic": "4*K*H*B*M*N FLOP per launch",
-        "second_ceiling": ex2_roofline(achieved, torch.cuda.get_device_properties(dev).multi_processor_count, 64),
+        "second_ceiling": ex2_roofline(achieved,
+                                       torch.cuda.get_device_properties(dev).multi_processor_count,
+                                       64, clocks.get("sm_mhz")),
     }
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -536,13 +541,32 @@ def measure_backward(mea, p, dev, stream, tc_peak, iters=5):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     B, M, Hq, K = q.shape
     ws = torch.empty(mea.lib.mea_bwd_workspace_size(B, M, Hq, K), dtype=torch.uint8, device=dev)
-    ms = _time(lambda: mea.mea_bwd(q, k, v, out, dout, lse, bias=p.bias, scale=p.scale,
-                                   alibi=p.alibi, dq=dq, dk=dk, dv=dv, workspace=ws, **kw),
-               stream, iters)
+    def run(stages=7):
+        mea.mea_bwd(q, k, v, out, dout, lse, bias=p.bias, scale=p.scale, alibi=p.alibi, dq=dq,
+                    dk=dk, dv=dv, workspace=ws, stages=stages, **kw)
+
+    ms = _time(run, stream, iters)
+    # The three launches one by one (mea_bwd_stages), with events between them.
+    names = ("bwd_prep", "bwd_kernel", "bwd_dq_out")
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
+    for e in evs:
+        e[0].record(stream)
+        for i, st in enumerate((1, 2, 4)):
+            run(st)
+            e[i + 1].record(stream)
+    torch.cuda.synchronize()
+    stage_ms = {n: round(statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs), 4)
+                for i, n in enumerate(names)}
     f = 2.5 * prefill_flops(p)
     tf = f / (ms * 1e-3) / 1e12
+    tf_main = f / (stage_ms["bwd_kernel"] * 1e-3) / 1e12
     return {"workload": "bwd_" + p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
             "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor",
+            "stage_ms": stage_ms, "bwd_kernel_tflops": round(tf_main, 1),
+            "bwd_kernel_frac": round(tf_main / tc_peak, 4),
             "kernel": "bwd_kernel (tcgen05, TMA; dq by TMA tensor reductions)"}
 
 
@@ -624,6 +648,8 @@ PROFILE_CASES = {
     "fwd_sweep_all": lambda: ("sweep", None),
     "fwd_sweep_m2048": lambda: ("fwd", synth.noncausal_sweep(2048)),
     "fwd_gqa_alibi_m2048": lambda: ("fwd", synth.gqa_alibi_causal(M=2048, B=2)),
+    "fwd_gqa_alibi_full": lambda: ("fwd", synth.gqa_alibi_causal()),
+    "bwd_gqa_alibi_full": lambda: ("bwd", synth.gqa_alibi_causal()),
     "fwd_varlen": lambda: ("fwd", synth.varlen_causal()),
     "bwd_m2048": lambda: ("bwd", synth.noncausal_sweep(2048)),
     "block_sparse_m2048": lambda: ("sparse", synth.block_sparse_noncausal(2048)),

@@ -135,6 +135,13 @@ int mea_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
  * lse = -inf.  The cache is split into fixed chunks processed in parallel; the
  * partial (max, sum, output) states are merged exactly by their log-sum-exp.
  *
+ * Device-side errors: a sequence whose offsets are inconsistent (n_b < 0, a
+ * negative start, rows past cache_rows, or n_b > max_kv_len rounded up to the
+ * split size), or one whose bounded pipeline wait gave up, gets out = 0 and
+ * lse = NaN for all its heads, and the device status word (mea_read_device_status)
+ * records MEA_ERR_INVALID_ARG or MEA_ERR_DEVICE_TIMEOUT; the other sequences
+ * are unaffected.  No result is ever assembled from another call's partials.
+ *
  * workspace: DEVICE scratch of at least mea_decode_workspace_size(...) bytes,
  * 256-byte aligned, owned by the caller; its contents need no initialisation
  * and are garbage afterwards.  Calls that share a workspace must not overlap.
@@ -168,9 +175,10 @@ int mea_decode(const void* q, const void* k_cache, const void* v_cache,
  * Notes for callers:
  *  - Every GPU that loads this library holds the 32 MiB array until the
  *    process exits.
- *  - The first call on each device looks up the array's device address with
- *    that device current, and caches it.  Make that first call before any stream
- *    capture begins.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, which allocates nothing); the first call on a
+ *    device also loads the library's kernels there, so make it before any
+ *    stream capture begins.
  *  - All calls on a device share the one array, which keeps the last call's
  *    contents.  Nothing in it has to start at zero: every partial a call reads,
  *    the same call has written first.  Calls whose executions overlap on the GPU
@@ -289,6 +297,30 @@ int mea_bwd(const void* q, const void* k, const void* v, const void* out, const 
             int num_seqs, int max_seqlen_q, int max_seqlen_k,
             int alibi, float scale, void* workspace, size_t workspace_bytes,
             cudaStream_t stream);
+
+/*
+ * mea_bwd_stages -- mea_bwd restricted to some of its three launches, in order:
+ *   MEA_BWD_PREP (1)  D_i = <dout_i, out_i> and a zeroed fp32 dq accumulator,
+ *                     both in the workspace;
+ *   MEA_BWD_MAIN (2)  dk, dv and the dq accumulation (the score recomputation);
+ *   MEA_BWD_DQ   (4)  the accumulator rounded into dq.
+ * `stages` is a bitwise OR of these (nonzero, else MEA_ERR_INVALID_ARG); the
+ * other arguments are those of mea_bwd.  Calling the three stages one by one on
+ * one stream, with the same arguments and workspace, computes exactly what one
+ * mea_bwd call computes; it lets a caller time or overlap the stages separately.
+ * A stage reads the workspace its predecessor wrote, so a stage run alone is
+ * meaningful only after its predecessors ran with the same workspace.
+ */
+enum { MEA_BWD_PREP = 1, MEA_BWD_MAIN = 2, MEA_BWD_DQ = 4 };
+
+int mea_bwd_stages(const void* q, const void* k, const void* v, const void* out,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   int B, int M, int N, int Hq, int Hkv, int K,
+                   mea_dtype_t dtype, mea_bias_t bias,
+                   const int32_t* seqstart_q, const int32_t* seqstart_k,
+                   int num_seqs, int max_seqlen_q, int max_seqlen_k,
+                   int alibi, float scale, void* workspace, size_t workspace_bytes,
+                   int stages, cudaStream_t stream);
 
 /* Number of key/value rows one decode split covers (the unit of parallelism). */
 int mea_decode_chunk(void);

@@ -423,13 +423,15 @@ extern "C" size_t mea_bwd_workspace_size(int B, int M, int Hq, int K) {
   return align256(rows * K * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* out,
-                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
-                       int M, int N, int Hq, int Hkv, int K, mea_dtype_t dtype, mea_bias_t bias,
-                       const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
-                       int max_seqlen_q, int max_seqlen_k, int alibi, float scale,
-                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+extern "C" int mea_bwd_stages(const void* q, const void* k, const void* v, const void* out,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int M, int N, int Hq, int Hkv, int K, mea_dtype_t dtype,
+                              mea_bias_t bias, const int32_t* seqstart_q,
+                              const int32_t* seqstart_k, int num_seqs, int max_seqlen_q,
+                              int max_seqlen_k, int alibi, float scale, void* workspace,
+                              size_t workspace_bytes, int stages, cudaStream_t stream) {
   (void)max_seqlen_q;
+  if (stages <= 0 || stages > 7) return MEA_ERR_INVALID_ARG;
   if (B < 0 || M < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return MEA_ERR_INVALID_ARG;
   if (dtype != MEA_F16 && dtype != MEA_BF16) return MEA_ERR_INVALID_ARG;
   if (bias < MEA_BIAS_NONE || bias > MEA_BIAS_BLOCKDIAG_CAUSAL) return MEA_ERR_INVALID_ARG;
@@ -499,11 +501,23 @@ extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* 
   L.mask = static_cast<int>(bias);
   L.alibi = alibi != 0;
   // The kernel writes every key row of every sequence; rows no sequence owns
-  // (packed batches) and the no-query case are zeroed here.
-  if (N > 0 && (M == 0 || packed) &&
+  // (packed batches) and the no-query case are zeroed here (with the main stage).
+  if ((stages & MEA_BWD_MAIN) && N > 0 && (M == 0 || packed) &&
       (cudaMemsetAsync(dk, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess ||
        cudaMemsetAsync(dv, 0, static_cast<size_t>(B) * N * Hkv * K * 2, stream) != cudaSuccess))
     return MEA_ERR_CUDA;
   if (M == 0) return MEA_OK;
-  return mea::launch_bwd(L, stream) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+  return mea::launch_bwd(L, stream, stages) == cudaSuccess ? MEA_OK : MEA_ERR_CUDA;
+}
+
+extern "C" int mea_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                       int M, int N, int Hq, int Hkv, int K, mea_dtype_t dtype, mea_bias_t bias,
+                       const int32_t* seqstart_q, const int32_t* seqstart_k, int num_seqs,
+                       int max_seqlen_q, int max_seqlen_k, int alibi, float scale,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return mea_bwd_stages(q, k, v, out, dout, lse, dq, dk, dv, B, M, N, Hq, Hkv, K, dtype, bias,
+                        seqstart_q, seqstart_k, num_seqs, max_seqlen_q, max_seqlen_k, alibi,
+                        scale, workspace, workspace_bytes,
+                        MEA_BWD_PREP | MEA_BWD_MAIN | MEA_BWD_DQ, stream);
 }

@@ -632,9 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool BF16, int MASK, bool ALIBI>
 cudaError_t launch_main(const BwdLaunch& L, cudaStream_t stream) {
-  auto kern = bwd_kernel<D, BF16, MASK, ALIBI>;
+  constexpr auto kern = bwd_kernel<D, BF16, MASK, ALIBI>;
   const int smem = BwdCfg<D>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_smem_once<kern>(smem);
   if (e != cudaSuccess) return e;
   const BwdArgs& a = L.args;
   dim3 grid(a.num_kblocks, a.Hkv, a.num_units);
@@ -643,14 +643,17 @@ cudaError_t launch_main(const BwdLaunch& L, cudaStream_t stream) {
 }
 
 template <int D, bool BF16>
-cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream) {
+cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream, int stages) {
   const BwdArgs& a = L.args;
   const long long rows = static_cast<long long>(a.B) * a.M * a.Hq;
   if (rows <= 0) return cudaSuccess;
-  bwd_prep_kernel<D, BF16><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  if (a.num_kblocks > 0 && a.N > 0) {
+  cudaError_t e = cudaSuccess;
+  if (stages & 1) {
+    bwd_prep_kernel<D, BF16><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if ((stages & 2) && a.num_kblocks > 0 && a.N > 0) {
     switch (L.mask * 2 + (L.alibi ? 1 : 0)) {
       case 0: e = launch_main<D, BF16, 0, false>(L, stream); break;
       case 1: e = launch_main<D, BF16, 0, true>(L, stream); break;
@@ -664,6 +667,7 @@ cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream) {
     }
     if (e != cudaSuccess) return e;
   }
+  if (!(stages & 4)) return cudaSuccess;
   const long long pairs = rows * D / 2;
   const long long blocks = std::min((pairs + 255) / 256, 148LL * 16);
   bwd_dq_out_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a);
@@ -682,11 +686,13 @@ extern "C" int mea_bwd_trace_read(long long* host, int n) {
 
 int bwd_query_block(int head_dim) { return head_dim == 128 ? BwdCfg<128>::BM : BwdCfg<64>::BM; }
 
-cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t stream) {
+cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t stream, int stages) {
   if (L.head_dim == 64)
-    return L.bf16 ? launch_all<64, true>(L, stream) : launch_all<64, false>(L, stream);
+    return L.bf16 ? launch_all<64, true>(L, stream, stages)
+                  : launch_all<64, false>(L, stream, stages);
   if (L.head_dim == 128)
-    return L.bf16 ? launch_all<128, true>(L, stream) : launch_all<128, false>(L, stream);
+    return L.bf16 ? launch_all<128, true>(L, stream, stages)
+                  : launch_all<128, false>(L, stream, stages);
   return cudaErrorInvalidValue;
 }
 

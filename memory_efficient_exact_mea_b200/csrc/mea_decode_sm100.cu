@@ -19,7 +19,6 @@
 //   * a second kernel merges the chunk partials exactly by their log-sum-exp.
 #include <math.h>
 
-#include <mutex>
 
 #include "mea.h"
 #include "mea_internal.h"
@@ -296,9 +295,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
   }
   __syncthreads();
-  if (*abort_flag) return;
-
   const int G = a.group;
+  if (*abort_flag) {
+    // A wait gave up (the status word holds the timeout): mark this split's
+    // partials as failed so the merge writes no result built from them.
+    if (threadIdx.x < G) {
+      const long long row = static_cast<long long>(b) * a.Hq + kvh * G + threadIdx.x;
+      a.part_lse[row * a.max_splits + split] = __int_as_float(0x7fc00000);
+    }
+    return;
+  }
+
   for (int idx = threadIdx.x; idx < G * D; idx += kThreads) {
     const int g = idx / D, d = idx - g * D;
     float mx = neg_inf();
@@ -327,15 +334,36 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   const int lane = threadIdx.x & 31;
   if (row >= a.B * a.Hq) return;
   const int b = row / a.Hq;
-  const int n = a.kv_seqstart[b + 1] - a.kv_seqstart[b];
-  if (lane == 0 && row % a.Hq == 0 &&
-      (n < 0 || static_cast<long long>(n) > static_cast<long long>(a.max_splits) * kDecodeChunk))
-    record_error(a.status, kErrInvalidArg);
-  const int ns = n <= 0 ? 0 : min((n + kDecodeChunk - 1) / kDecodeChunk, a.max_splits);
+  const int t0 = a.kv_seqstart[b];
+  const int n = a.kv_seqstart[b + 1] - t0;
+  uint16_t* out = static_cast<uint16_t*>(a.out) + static_cast<long long>(row) * D;
+  // The partial kernel's checks of this sequence's offsets: a sequence it
+  // skipped has no partials, so its rows get out = 0 and lse = NaN (and the
+  // status word the error) rather than whatever the workspace held.
+  if (n < 0 || t0 < 0 || t0 + n > a.cache_rows ||
+      static_cast<long long>(n) > static_cast<long long>(a.max_splits) * kDecodeChunk) {
+    if (lane == 0 && row % a.Hq == 0) record_error(a.status, kErrInvalidArg);
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) out[lane + 32 * i] = 0;
+    if (lane == 0 && a.lse != nullptr) a.lse[row] = __int_as_float(0x7fc00000);
+    return;
+  }
+  const int ns = n <= 0 ? 0 : (n + kDecodeChunk - 1) / kDecodeChunk;
   const float* pl = a.part_lse + static_cast<long long>(row) * a.max_splits;
   const float* po = a.part_o + static_cast<long long>(row) * a.max_splits * D;
   float mx = neg_inf();
-  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, pl[s]);
+  bool failed = false;  // a split whose partial kernel gave up
+  for (int s = lane; s < ns; s += 32) {
+    const float x = pl[s];
+    failed |= x != x;
+    mx = fmaxf(mx, x);
+  }
+  if (__any_sync(0xffffffffu, failed)) {
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) out[lane + 32 * i] = 0;
+    if (lane == 0 && a.lse != nullptr) a.lse[row] = __int_as_float(0x7fc00000);
+    return;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   const float msub = (mx == neg_inf()) ? 0.f : mx;
@@ -350,7 +378,6 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
     for (int i = 0; i < D / 32; ++i) o[i] = fmaf(w, po[s * D + lane + 32 * i], o[i]);
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  uint16_t* out = static_cast<uint16_t*>(a.out) + static_cast<long long>(row) * D;
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) {
     const float v = o[i] * inv;
@@ -370,9 +397,9 @@ template <int D, bool BF16, bool ALIBI>
 cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t stream) {
   const DecodeArgs& a = L.args;
   if (a.max_splits > 0 && a.B > 0) {
-    auto kern = decode_partial_kernel<D, BF16, ALIBI>;
+    constexpr auto kern = decode_partial_kernel<D, BF16, ALIBI>;
     const int smem = DSmem<D>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_once<kern>(smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.max_splits, a.Hkv, a.B);
     kern<<<grid, kThreads, smem, stream>>>(L.tmK, L.tmV, a);
@@ -396,29 +423,20 @@ cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t stream) {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per device
-constexpr int kMaxDevices = 64;
 
 // Every device that loads this library holds this array until the process exits.
 static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 // Device address of g_decode_scratch on the current device.  Host code cannot use
 // the symbol itself (on the host it names a stand-in, not device memory), so the
-// address is looked up once per device, with that device current, and cached.
+// address is looked up on every call, with the caller's device current (the
+// lookup is cheap, and a cached address would go stale if the device's context
+// were torn down and created again).
 cudaError_t noalloc_scratch(void** ptr) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  static std::mutex mu;
-  static void* cached[kMaxDevices] = {};
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    cached[dev] = p;
-  }
-  *ptr = cached[dev];
+  *ptr = p;
   return cudaSuccess;
 }
 

@@ -6,7 +6,27 @@
 #include <cuda_runtime_api.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace mea {
+
+// Raises kernel KERN's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute lasts as long as the device's
+// context); later calls only test a bit.  If the context is destroyed and
+// created again (cudaDeviceReset), the bit stays set and the kernel's launch
+// then fails with an error status instead of running.
+template <auto KERN>
+cudaError_t set_smem_once(int bytes) {
+  static std::atomic<unsigned long long> done{0};  // bit d: done on device d (d < 64)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Prefill: one CTA computes two 128-row query tiles of one (sequence, head).
 constexpr int kFwdRowsPerCta = 256;
@@ -109,7 +129,9 @@ struct BwdLaunch {
   bool alibi;
 };
 
-cudaError_t launch_bwd(const BwdLaunch& launch, cudaStream_t stream);
+// stages: bit 0 the D / accumulator preparation, bit 1 the main kernel, bit 2
+// the dq conversion (the three launches of one backward, in that order).
+cudaError_t launch_bwd(const BwdLaunch& launch, cudaStream_t stream, int stages = 7);
 
 // Query rows per step of the backward kernel for head dimension 64 or 128.
 int bwd_query_block(int head_dim);
