@@ -325,7 +325,7 @@ def run_ours(args, rank, world, local):
         also["gqa_alibi_causal"] = measure_prefill(mea, synth.gqa_alibi_causal(), dev, stream,
                                                    tc_peak)
         also["causal_small"] = measure_prefill(mea, synth.causal_small(), dev, stream, tc_peak,
-                                               iters=50)
+                                               iters=50, host_paths=True)
         also["decode"] = measure_decode(mea, synth.decode_step(), dev, stream, hbm_peak)
         also["chunk_prefill"] = measure_chunk(mea, synth.chunk_prefill(), dev, stream, tc_peak)
         bs_p, bs_mask = synth.block_sparse_noncausal()
@@ -475,7 +475,7 @@ def _time(fn, stream, iters, warmup=3):
     return e0.elapsed_time(e1) / iters
 
 
-def measure_prefill(mea, p, dev, stream, tc_peak, iters=10):
+def measure_prefill(mea, p, dev, stream, tc_peak, iters=10, host_paths=False):
     q, k, v = p.q.to(dev), p.k.to(dev), p.v.to(dev)
     kw = {}
     if p.seq_lens_q is not None:
@@ -488,8 +488,27 @@ def measure_prefill(mea, p, dev, stream, tc_peak, iters=10):
                                    lse=lse, **kw), stream, iters)
     f = prefill_flops(p)
     tf = f / (ms * 1e-3) / 1e12
-    return {"workload": p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
-            "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor"}
+    r = {"workload": p.name, "ms": round(ms, 4), "tflops": round(tf, 1),
+         "frac": round(tf / tc_peak, 4), "flop": f, "bound": "tensor"}
+    if host_paths:
+        # Calls back to back on one stream, three ways: the plain binding call
+        # above (Python marshalling every call), a prepared call (the C entry
+        # point only), and prepared calls captured in a CUDA graph (launch gaps
+        # only: close to the kernel's own time).
+        call = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, out=out, lse=lse,
+                           prepare=True, **kw)
+        r["ms_prepared"] = round(_time(call, stream, iters), 4)
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):  # prepared on the capturing stream
+            gcall = mea.mea_fwd(q, k, v, bias=p.bias, scale=p.scale, alibi=p.alibi, out=out,
+                                lse=lse, prepare=True, **kw)
+            for _ in range(20):
+                gcall()
+        torch.cuda.synchronize()
+        r["ms_graph"] = round(_time(g.replay, torch.cuda.current_stream(), 5) / 20, 4)
+        r["host_note"] = "ms: plain binding call; ms_prepared: marshalled once; ms_graph: 20 calls per CUDA graph"
+    return r
 
 
 def measure_block_sparse(mea, p, mask, dev, stream, tc_peak, iters=10):

@@ -22,7 +22,7 @@ import torch
 
 __all__ = ["mea_fwd", "mea_fwd_block_sparse", "mea_prefill_chunk", "mea_bwd", "mea_decode",
            "mea_decode_workspace_size", "mea_decode_chunk", "read_device_status", "status_string",
-           "MeaError", "BIAS", "BWD_PREP", "BWD_MAIN", "BWD_DQ", "LIB_PATH", "lib"]
+           "MeaError", "PreparedCall", "BIAS", "BWD_PREP", "BWD_MAIN", "BWD_DQ", "LIB_PATH", "lib"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmea.so")
 
@@ -109,6 +109,7 @@ def _check(fn, rc):
 _STRIDES: dict = {}  # (sb, sm, sh) -> ctypes int64[3], reused across calls (read-only)
 
 
+
 def _bmhk_strides(t: torch.Tensor, name: str):
     st = t.stride()
     if len(st) != 4:
@@ -148,10 +149,29 @@ def _grouped_views(q, k, v, out):
     return q4, kv4(k, "k"), kv4(v, "v"), o4
 
 
+class PreparedCall:
+    """One C-ABI call with every argument marshalled once, for launching the same
+    computation again and again (a serving or training loop whose buffers stay
+    put): calling it only runs the C entry point, on the stream chosen when it
+    was prepared.  It keeps the tensors it points into alive.  `outputs` holds
+    what the call writes."""
+
+    __slots__ = ("_fn", "_args", "_name", "_keep", "outputs")
+
+    def __init__(self, fn, args, name, keep, outputs):
+        self._fn, self._args, self._name, self._keep, self.outputs = fn, args, name, keep, outputs
+
+    def __call__(self):
+        rc = self._fn(*self._args)
+        if rc != 0:
+            raise MeaError(self._name, rc)
+        return self.outputs
+
+
 def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool = False,
             seqstart_q=None, seqstart_k=None, max_seqlen_q: int | None = None,
             max_seqlen_k: int | None = None, out=None, lse=None, return_lse: bool = True,
-            stream=None):
+            stream=None, prepare: bool = False):
     """Attention forward.  q [B,M,Hq,K], k/v [B,N,Hkv,K] (fp16/bf16, CUDA) ->
     (out [B,M,Hq,K], lse [B,Hq,M] fp32 or None).
 
@@ -164,8 +184,14 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
     [B,N,G,H,K] with stride 0) is the same call with Hq = G*H query heads and
     Hkv = G key/value heads, query head g*H + r reading key/value head g; out is
     returned as [B,M,G,H,K] and lse as [B,G*H,M].
+
+    prepare=True launches nothing and returns a PreparedCall instead: each call
+    of it runs this forward again on the same buffers (its outputs are
+    (out, lse)), with no Python-side argument handling.
     """
     if q.dim() == 5:
+        if prepare:
+            raise ValueError("prepare=True takes the 4-D layout")
         shape5 = tuple(q.shape)
         q, k, v, out4 = _grouped_views(q, k, v, out)
         o, l = mea_fwd(q, k, v, bias, scale, alibi, seqstart_q, seqstart_k, max_seqlen_q,
@@ -201,12 +227,15 @@ def mea_fwd(q, k, v, bias: str = "none", scale: float | None = None, alibi: bool
     else:
         seqstart_q = seqstart_k = None
         max_seqlen_q = max_seqlen_k = 0
-    rc = lib.mea_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, M, N, Hq, Hkv, K,
-                     _bmhk_strides(q, "q"), _bmhk_strides(k, "k"), _bmhk_strides(v, "v"),
-                     _bmhk_strides(out, "out"), _DTYPE[q.dtype], kind, _ptr(seqstart_q),
-                     _ptr(seqstart_k), ns, int(max_seqlen_q), int(max_seqlen_k), int(bool(alibi)),
-                     scale, _stream(stream, q.device))
-    _check("mea_fwd", rc)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, M, N, Hq, Hkv, K,
+            _bmhk_strides(q, "q"), _bmhk_strides(k, "k"), _bmhk_strides(v, "v"),
+            _bmhk_strides(out, "out"), _DTYPE[q.dtype], kind, _ptr(seqstart_q), _ptr(seqstart_k),
+            ns, int(max_seqlen_q), int(max_seqlen_k), int(bool(alibi)), scale,
+            _stream(stream, q.device))
+    if prepare:
+        return PreparedCall(lib.mea_fwd, args, "mea_fwd",
+                            (q, k, v, out, lse, seqstart_q, seqstart_k), (out, lse))
+    _check("mea_fwd", lib.mea_fwd(*args))
     return out, lse
 
 

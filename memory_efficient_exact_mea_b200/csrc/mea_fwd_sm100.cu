@@ -130,12 +130,22 @@ __device__ long long g_cta_trace[kCtaTraceMax * 8];
 // region is shifted back to end at the region's end (its first columns, seen by
 // an earlier tile or before row 0, are masked), so no row beyond a sequence's
 // valid rows is ever loaded.
-// Persistent instances: one CTA per SM walks the units blockIdx.x, + gridDim.x, ...
-// with every pipeline counter running on across units, so the next unit's Q, K/V
-// and first Q.K^T overlap the current unit's last steps and output epilogue.
-// Dense, unpacked, non-causal K = 64 fp16 without ALiBi (units of equal length).
+// Persistent instances (every instance without a block mask or a cache): one CTA
+// per SM walks several units, with every pipeline counter running on across
+// units, so the next unit's Q, K/V and first Q.K^T overlap the current unit's
+// last steps and output epilogue.  The units are dealt out in a fixed order
+// (round k of CTA c takes rank k * gridDim.x + c, or + gridDim.x - 1 - c in odd
+// rounds), so the heaviest units of a causal launch, which come first in rank
+// order, are spread over every SM.
 template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
-constexpr bool kPersistent = D == 64 && !BF16 && MASK == 0 && !ALIBI && MODE == kModeDense;
+constexpr bool kPersistent = MODE == kModeDense;
+
+// Q buffers (two query tiles each): persistent instances at K = 64 double-buffer
+// Q, so the next unit's Q lands during this unit's key loop; at K = 128 (no
+// shared memory to spare) the one buffer is reloaded once this unit's last
+// Q.K^T has completed.
+template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
+constexpr int kQBuffers = (kPersistent<D, BF16, MASK, ALIBI, MODE> && D == 64) ? 2 : 1;
 
 template <int D, bool BF16, int MASK, bool ALIBI, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -145,8 +155,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool SPARSE = (MODE == kModeSparse);
   constexpr bool kCache = (MODE == kModeCache);
   constexpr bool kPersist = kPersistent<D, BF16, MASK, ALIBI, MODE>;
-  constexpr int QB = kPersist ? 2 : 1;
-  using L = Smem<D, QB>;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
   constexpr bool kSplitP = BF16;  // P.V as (P_hi + P_lo).V for bf16
@@ -154,6 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // = 512), so S_t is free as soon as the softmax has read it and the next
   // Q.K^T of the same tile runs during its softmax.  Otherwise P is written over S.
   constexpr bool kSepP = (D == 64) && !BF16;
+  constexpr int QB = kQBuffers<D, BF16, MASK, ALIBI, MODE>;
+  using L = Smem<D, QB>;
   // Softmax tile body specialised separately for masked and unmasked tiles.
   constexpr bool kTileCopies = !ALIBI && MODE == kModeDense && !kPacked;
   constexpr uint32_t kColP = kSepP ? 2 * kBN : 0;          // + t * (kSepP ? kBN/2 : kBN)
@@ -182,104 +192,143 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   if (threadIdx.x == 0) MEA_CTA_AT(0);
 
-  // ---- which (query block, head, batch or sequence) this CTA owns ----------
-  // The query block varies fastest, so the blocks of one (head, batch) -- and
-  // the heads sharing a key/value head -- run together and read each K/V tile
-  // from L2 instead of DRAM.  Under a causal mask the longest rows go first.
-  int mb = blockIdx.x % a.num_mblocks;
-  const int rem = blockIdx.x / a.num_mblocks;
-  int h = rem % a.Hq;
-  int unit = rem / a.Hq;
-  if (kCausal) mb = a.num_mblocks - 1 - mb;
-  int kvh = h / a.group;
-
-  int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, bidx = unit;
-  if constexpr (kPacked) {
-    q0 = a.seqstart_q[unit];
-    q_len = a.seqstart_q[unit + 1] - q0;
-    k0 = a.seqstart_k[unit];
-    k_len = a.seqstart_k[unit + 1] - k0;
-    bidx = 0;
-    const bool bad = q_len < 0 || k_len < 0 || q0 < 0 || k0 < 0 || q0 + q_len > a.M ||
-                     k0 + k_len > a.N || (mb == a.num_mblocks - 1 &&
-                                          q_len > a.num_mblocks * kFwdRowsPerCta);
-    if (bad) {
-      if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
-      return;
-    }
-  }
+  // ---- units: (query block, head, batch or sequence) ------------------------
+  // A unit is two 128-row query tiles of one (head, batch or sequence); rank r
+  // numbers the units.  Without a causal mask the query block varies fastest,
+  // so the blocks of one (head, batch) -- and the heads sharing a key/value
+  // head -- run together and read each K/V tile from L2 instead of DRAM.  Under
+  // a causal mask a unit's work grows with its query block, so the ranks go by
+  // query block, last (longest rows) first, with the heads fastest: the longest
+  // units of the whole launch start first.
+  const int n_ranks = a.num_mblocks * a.Hq * a.num_units;
+  int mb = 0, h = 0, unit = 0, kvh = 0, bidx = 0, m_base = 0;
+  int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, off = 0;
   int past = 0;  // cache mode: rows cached before this chunk
-  if constexpr (kCache) {
-    past = a.cache_len[unit];
-    q_len = a.q_lens ? a.q_lens[unit] : a.M;
-    if (past < 0 || q_len < 0 || q_len > a.M || past > a.cap - q_len) {
-      if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
-      return;
+  int n_past_tiles = 0, n_new_tiles = 0;
+  int nt_tile[2] = {0, 0};  // key tiles each query tile computes
+  int nt = 0;               // key tiles loaded (the larger of the two)
+  const uint8_t* mrow0 = nullptr;  // block-sparse: the two query tiles' mask rows
+  const uint8_t* mrow1 = nullptr;
+  // Moves every per-unit value to unit `rank`.  Returns 0 if the unit's sequence
+  // offsets are invalid (the status word records it; nothing to do), 1 if the
+  // unit has no query rows, 2 if it has rows to compute.
+  auto set_unit = [&](int rank) -> int {
+    if constexpr (kCausal) {
+      const int per = a.Hq * a.num_units;
+      const int level = rank / per;
+      const int rem = rank - level * per;
+      h = rem % a.Hq;
+      unit = rem / a.Hq;
+      mb = a.num_mblocks - 1 - level;
+    } else {
+      mb = rank % a.num_mblocks;
+      const int rem = rank / a.num_mblocks;
+      h = rem % a.Hq;
+      unit = rem / a.Hq;
     }
-    k_len = past + q_len;
-    // The append: the CTAs of one (sequence, kv head) -- its query heads times
-    // its query blocks -- each copy an equal share of the new rows.
-    const int slices = a.group * a.num_mblocks;
-    const int slice = (h % a.group) * a.num_mblocks + static_cast<int>(blockIdx.x % a.num_mblocks);
-    const long long r0 = static_cast<long long>(q_len) * slice / slices;
-    const long long r1 = static_cast<long long>(q_len) * (slice + 1) / slices;
-    constexpr int kPieces = D / 8;  // 16-byte pieces per row
-    for (long long e = threadIdx.x; e < (r1 - r0) * kPieces * 2; e += kThreads) {
-      const int kv = static_cast<int>(e & 1);
-      const long long r = r0 + (e >> 1) / kPieces;
-      const int c = static_cast<int>((e >> 1) % kPieces);
-      const long long* ns = kv ? a.vn_s : a.kn_s;
-      const long long* cs = kv ? a.vc_s : a.kc_s;
-      const uint4* src = reinterpret_cast<const uint4*>(
-          static_cast<const uint16_t*>(kv ? a.v_new : a.k_new) + unit * ns[0] + r * ns[1] +
-          kvh * ns[2] + c * 8);
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(kv ? a.v_cache : a.k_cache) +
-                                            unit * cs[0] + (past + r) * cs[1] + kvh * cs[2] +
-                                            c * 8);
-      *dst = *src;
-    }
-  }
-  int m_base = mb * kFwdRowsPerCta;
-  if (m_base >= q_len) return;
-  const int off = k_len - q_len;  // bottom-right causal alignment
-
-  // Key tiles each query tile needs.  Cache mode: the past tiles (all visible)
-  // then the new tiles (up to the diagonal under a causal mask).
-  const int n_past_tiles = kCache ? (past + kBN - 1) / kBN : 0;
-  const int n_new_tiles = kCache ? (q_len + kBN - 1) / kBN : 0;
-  int nt_tile[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int mt = m_base + t * kBM;
-    int nkeys = 0;
-    if (mt < q_len) {
-      nkeys = k_len;
-      if (kCausal) nkeys = min(k_len, max(0, mt + kBM + off));
-    }
-    nt_tile[t] = (nkeys + kBN - 1) / kBN;
-    if constexpr (kCache) {
-      const int nn = mt < q_len ? (kCausal ? min(q_len, mt + kBM) : q_len) : 0;
-      nt_tile[t] = mt < q_len ? n_past_tiles + (nn + kBN - 1) / kBN : 0;
-    }
-  }
-  int nt = max(nt_tile[0], nt_tile[1]);
-
-  // Units this CTA runs: blockIdx.x, + gridDim.x, ... below n_units (persistent
-  // instances), or just its own.  next_unit() moves the per-unit values to unit
-  // cu (persistent instances only: dense, unpacked, non-causal).
-  const int n_units = kPersist ? a.num_mblocks * a.Hq * a.num_units : static_cast<int>(gridDim.x);
-  auto next_unit = [&](int cu) {
-    mb = cu % a.num_mblocks;
-    const int r = cu / a.num_mblocks;
-    h = r % a.Hq;
-    unit = r / a.Hq;
     kvh = h / a.group;
     bidx = unit;
+    if constexpr (kPacked) {
+      q0 = a.seqstart_q[unit];
+      q_len = a.seqstart_q[unit + 1] - q0;
+      k0 = a.seqstart_k[unit];
+      k_len = a.seqstart_k[unit + 1] - k0;
+      bidx = 0;
+      const bool bad = q_len < 0 || k_len < 0 || q0 < 0 || k0 < 0 || q0 + q_len > a.M ||
+                       k0 + k_len > a.N || (mb == a.num_mblocks - 1 &&
+                                            q_len > a.num_mblocks * kFwdRowsPerCta);
+      if (bad) {
+        if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
+        return 0;
+      }
+    }
+    if constexpr (kCache) {
+      past = a.cache_len[unit];
+      q_len = a.q_lens ? a.q_lens[unit] : a.M;
+      if (past < 0 || q_len < 0 || q_len > a.M || past > a.cap - q_len) {
+        if (threadIdx.x == 0) record_error(a.status, kErrInvalidArg);
+        return 0;
+      }
+      k_len = past + q_len;
+    }
     m_base = mb * kFwdRowsPerCta;
+    if (m_base >= q_len) return 1;
+    off = k_len - q_len;  // bottom-right causal alignment
+    // Key tiles each query tile needs.  Cache mode: the past tiles (all visible)
+    // then the new tiles (up to the diagonal under a causal mask).
+    n_past_tiles = kCache ? (past + kBN - 1) / kBN : 0;
+    n_new_tiles = kCache ? (q_len + kBN - 1) / kBN : 0;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) nt_tile[t] = m_base + t * kBM < q_len ? (k_len + kBN - 1) / kBN : 0;
+    for (int t = 0; t < 2; ++t) {
+      const int mt = m_base + t * kBM;
+      int nkeys = 0;
+      if (mt < q_len) {
+        nkeys = k_len;
+        if (kCausal) nkeys = min(k_len, max(0, mt + kBM + off));
+      }
+      nt_tile[t] = (nkeys + kBN - 1) / kBN;
+      if constexpr (kCache) {
+        const int nn = mt < q_len ? (kCausal ? min(q_len, mt + kBM) : q_len) : 0;
+        nt_tile[t] = mt < q_len ? n_past_tiles + (nn + kBN - 1) / kBN : 0;
+      }
+    }
     nt = max(nt_tile[0], nt_tile[1]);
+    if constexpr (SPARSE) {
+      const long long base = unit * a.bm_sb + static_cast<long long>(h) * a.bm_sh;
+      mrow0 = a.block_mask + base + static_cast<long long>(2 * mb) * a.bm_nk;
+      mrow1 = mrow0 + a.bm_nk;
+    }
+    return 2;
   };
+  // Round k of this CTA: rank k * gridDim.x + c, or + gridDim.x - 1 - c in odd
+  // rounds (persistent instances); the CTA's own rank otherwise.
+  auto rank_of = [&](int k) -> int {
+    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return k * G + ((k & 1) ? G - 1 - c : c);
+  };
+  // Calls body() for each unit with query rows this CTA runs, in order, until
+  // body() returns false.  Every role walks the same units.
+  auto for_each_unit = [&](auto&& body) {
+    if constexpr (kPersist) {
+      for (int k = 0;; ++k) {
+        const int r = rank_of(k);
+        if (r >= n_ranks) return;
+        if (set_unit(r) != 2) continue;
+        if (!body(k)) return;
+      }
+    } else {
+      body(0);  // the CTA's unit, set below
+    }
+  };
+
+  if constexpr (!kPersist) {
+    const int st = set_unit(static_cast<int>(blockIdx.x));
+    if (st == 0) return;
+    if constexpr (kCache) {
+      // The append: the CTAs of one (sequence, kv head) -- its query heads times
+      // its query blocks -- each copy an equal share of the new rows.
+      const int slices = a.group * a.num_mblocks;
+      const int slice = (h % a.group) * a.num_mblocks + mb;
+      const long long r0 = static_cast<long long>(q_len) * slice / slices;
+      const long long r1 = static_cast<long long>(q_len) * (slice + 1) / slices;
+      constexpr int kPieces = D / 8;  // 16-byte pieces per row
+      for (long long e = threadIdx.x; e < (r1 - r0) * kPieces * 2; e += kThreads) {
+        const int kv = static_cast<int>(e & 1);
+        const long long r = r0 + (e >> 1) / kPieces;
+        const int c = static_cast<int>((e >> 1) % kPieces);
+        const long long* ns = kv ? a.vn_s : a.kn_s;
+        const long long* cs = kv ? a.vc_s : a.kc_s;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            static_cast<const uint16_t*>(kv ? a.v_new : a.k_new) + unit * ns[0] + r * ns[1] +
+            kvh * ns[2] + c * 8);
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(kv ? a.v_cache : a.k_cache) +
+                                              unit * cs[0] + (past + r) * cs[1] + kvh * cs[2] +
+                                              c * 8);
+        *dst = *src;
+      }
+    }
+    if (st == 1) return;
+  }
 
   // Key tile j: the row its copy starts at (in the cache or in the new rows),
   // the key position of its column 0 and its first column not already seen by
@@ -307,13 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Does query tile t compute key tile j?  Every role walks the key tiles in
   // the same order and skips those neither query tile needs; the barriers of a
   // query tile count only the key tiles that tile computes.
-  const uint8_t* mrow0 = nullptr;
-  const uint8_t* mrow1 = nullptr;
-  if constexpr (SPARSE) {
-    const long long base = unit * a.bm_sb + static_cast<long long>(h) * a.bm_sh;
-    mrow0 = a.block_mask + base + static_cast<long long>(2 * mb) * a.bm_nk;
-    mrow1 = mrow0 + a.bm_nk;
-  }
   auto uses = [&](int t, int j) -> bool {
     if (j >= nt_tile[t]) return false;
     if constexpr (SPARSE) return __ldg(t ? mrow1 + j : mrow0 + j) != 0;
@@ -324,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int qb = 0; qb < QB; ++qb) {
       mbar_init(&q_full[qb], 1);
-      mbar_init(&q_empty[qb], 2);  // one commit per MMA-issuing thread (separate-P layout)
+      mbar_init(&q_empty[qb], kSepP ? 2 : 1);  // one commit per MMA-issuing thread
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -360,50 +402,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // ===================== TMA producer =====================================
-    if (!kPersist && lane == 0 && nt > 0) {
-      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, q_full, c * 64, h,
-                      q0 + m_base + t * kBM, bidx);
-      int it = 0;
-      for (int j = 0; j < nt; ++j) {
-        if constexpr (SPARSE) {
-          if (!uses(0, j) && !uses(1, j)) continue;
-        }
-        const KeyTile kt = key_tile(j);
-        for (int kv = 0; kv < 2; ++kv, ++it) {
-          const int slot = it % S;
-          if (!mbar_wait(&kv_empty[slot], ((it / S) & 1) ^ 1, abort_flag, a.status)) break;
-          mbar_arrive_expect_tx(&kv_full[slot], L::kTileBytes);
-          const CUtensorMap* map = kv ? &tmV : &tmK;
-          if (kCache && kt.fresh) map = kv ? &tmVn : &tmKn;
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
-                        c * 64, kvh, kt.row, bidx);
-        }
-        if (*abort_flag) break;
-      }
-      // Let every copy this thread started land before the CTA can exit.
-      mbar_wait_drain(q_full, 0, a.status);
-      for (int i = max(0, it - S); i < it; ++i)
-        mbar_wait_drain(&kv_full[i % S], (i / S) & 1, a.status);
-    }
-    // Persistent instances: Q double-buffered, ring and unit counters run on.
-    if (kPersist && lane == 0 && nt > 0) {
-      int it = 0, iu = 0;  // K/V ring copies and units, over all units
-      bool ok = true;
-      for (int cu = blockIdx.x;; cu += gridDim.x) {
-        if (iu > 0) next_unit(cu);
+    // Per unit: its two Q tiles into Q buffer (unit count) % QB, then its K and V
+    // tiles through the ring; the ring and unit counters run on across units.
+    if (lane == 0) {
+      int it = 0, iu = 0;  // K/V ring copies and Q loads, over all units
+      for_each_unit([&](int) -> bool {
+        if (nt == 0) return true;  // rows that see no key: nothing to load
         const int qb = iu % QB;
         // The buffer's previous unit (QB units back) has finished its Q.K^T MMAs.
-        if (iu >= QB && !(ok = mbar_wait(&q_empty[qb], (iu / QB - 1) & 1, abort_flag, a.status)))
-          break;
+        if (iu >= QB && !mbar_wait(&q_empty[qb], (iu / QB - 1) & 1, abort_flag, a.status))
+          return false;
         mbar_arrive_expect_tx(&q_full[qb], 2 * L::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sQ + (2 * qb + t) * L::kTileBytes + c * L::kChunkBytes, &tmQ, &q_full[qb],
                         c * 64, h, q0 + m_base + t * kBM, bidx);
+        ++iu;
         for (int j = 0; j < nt; ++j) {
           if constexpr (SPARSE) {
             if (!uses(0, j) && !uses(1, j)) continue;
@@ -419,11 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
                           c * 64, kvh, kt.row, bidx);
           }
-          if (*abort_flag) break;
+          if (*abort_flag) return false;
         }
-        ++iu;
-        if (*abort_flag || cu + static_cast<int>(gridDim.x) >= n_units) break;
-      }
+        return *abort_flag == 0;
+      });
       // Let every copy this thread started land before the CTA can exit.
       for (int i = max(0, iu - QB); i < iu; ++i)
         mbar_wait_drain(&q_full[i % QB], (i / QB) & 1, a.status);
@@ -497,53 +510,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&kv_empty[vs]);
         return true;
       };
-      // Separate-P layout, one unit per CTA.
-      if (!kPersist && kSepP && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
-        bool ok = true, prev_used = false;
-        int li = 0, c = 0, prev_c = 0;
-        for (int j = 0; j < nt && ok; ++j) {
-          const bool used = uses(t, j);
-          if constexpr (SPARSE) {
-            if (!used && !uses(1 - t, j)) continue;
-          } else {
-            li = j;  // dense: every key tile is in the ring and a tile uses a prefix
-            c = j;
-          }
-          const int ks = (2 * li) % S;
-          if (!(ok = mbar_wait(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + t * 256 + li * 8 + 0);
-          if (used) {
-            if (c > 0) {  // the softmax has read the previous S_t out of TMEM
-              if (!(ok = mbar_wait(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
-              tc_fence_after();
-            }
-            issue_qk(t, ks, q_addr);
-            umma_commit(&s_full[t]);
-            MEA_TRACE_AT(1024 + t * 256 + li * 8 + 1);
-          }
-          umma_commit(&kv_empty[ks]);
-          if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c, prev_c > 0);
-          prev_used = used;
-          prev_c = c;
-          c += used ? 1 : 0;
-          ++li;
-        }
-        if constexpr (!SPARSE) li = nt;
-        if (ok && li > 0) pv_step(li - 1, prev_used, prev_c, prev_c > 0);
-      }
-      // Persistent instances (separate-P layout, several units per CTA): the stream
-      // stays one step behind for P.V over unit boundaries too, so the next unit's
-      // first Q.K^T goes out before this unit's last P.V.
-      if (kPersist && nt > 0) {
+      // Separate-P layout: one thread per query tile.  P.V stays one step behind
+      // Q.K^T, over unit boundaries too, so the next unit's first Q.K^T goes out
+      // before this unit's last P.V.
+      if constexpr (kSepP) {
         bool ok = true, prev_used = false, prev_acc = false;
         // li: key tiles in the ring, c: key tiles this query tile computed (its
-        // barrier phases), both over all units; li0, c0: their values at the unit's start.
-        int li = 0, c = 0, prev_c = 0, li0 = 0, c0 = 0, iu = 0;
-        for (int cu = blockIdx.x;; cu += gridDim.x, ++iu) {
-          if (iu > 0) next_unit(cu);
+        // barrier phases), both over all units; iu: units with keys so far.
+        int li = 0, c = 0, prev_c = 0, iu = 0;
+        for_each_unit([&](int) -> bool {
+          if (nt == 0) return true;
           const int qb = iu % QB;
-          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) break;
+          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
           const uint32_t q_buf = q_addr + 2 * qb * L::kTileBytes;
+          const int li0 = li, c0 = c;
           for (int j = 0; j < nt && ok; ++j) {
             const bool used = uses(t, j);
             if constexpr (SPARSE) {
@@ -576,81 +556,101 @@ __global__ void __launch_bounds__(kThreads, 1)
             li = li0 + nt;
             c = c0 + nt_tile[t];
           }
-          li0 = li;
-          c0 = c;
           // This unit's Q buffer is free once its Q.K^T MMAs have completed.
-          umma_commit(&q_empty[qb]);
-          if (!ok || cu + static_cast<int>(gridDim.x) >= n_units) break;
-        }
+          if constexpr (kPersist) umma_commit(&q_empty[qb]);
+          ++iu;
+          return ok;
+        });
         if (ok && li > 0) pv_step(li - 1, prev_used, prev_c, prev_acc);
       }
       // When P is written over S the chain softmax -> P.V -> Q.K^T of a tile is
       // serial, so one thread (warp 16) issues both tiles in the interleaved
       // order Q0.K_j, P1.V_{j-1}, Q1.K_j, P0.V_j, which keeps the two tiles half a
-      // step apart: one tile's softmax overlaps the other tile's MMAs.
-      if (!kSepP && tile == 0 && nt > 0 && mbar_wait(q_full, 0, abort_flag, a.status)) {
-        // li: key tiles in the ring; c0, c1: key tiles computed by query tile 0, 1.
-        int it = 0, vslot_prev = 0, li = 0, c0 = 0, c1 = 0, prev_c1 = 0;
-        bool ok = true, prev_u1 = false;
-        for (int j = 0; j < nt && ok; ++j) {
-          const bool u0 = uses(0, j), u1 = uses(1, j);
-          if constexpr (SPARSE) {
-            if (!u0 && !u1) continue;
-          } else {  // dense: every key tile is in the ring and each tile uses a prefix
-            li = j;
-            it = 2 * j;
-            c0 = j;
-            c1 = j;
-          }
-          const int kslot = it % S;
-          if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + li * 16 + 0);
-          ++it;
-          if (u0) {
-            issue_qk(0, kslot, q_addr);
-            MEA_TRACE_AT(1024 + li * 16 + 1);
-            umma_commit(&s_full[0]);
-          }
-          if (li >= 1) {
-            if (prev_u1) {
-              if (!(ok = mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status))) break;
-              MEA_TRACE_AT(1024 + li * 16 + 2);
-              tc_fence_after();
-              issue_pv(1, vslot_prev, prev_c1 > 0);
-              umma_commit(&o_done[1]);
+      // step apart: one tile's softmax overlaps the other tile's MMAs.  The P1.V
+      // lag runs on over unit boundaries: the next unit's Q0.K_0 goes out before
+      // this unit's last P1.V (S_0 is free once P0.V of the last step is issued,
+      // since the MMAs of one thread execute in issue order).
+      if (!kSepP && tile == 0) {
+        // li: key tiles in the ring; it: ring slots; c0, c1: key tiles computed by
+        // query tile 0, 1 (their barrier phases); all over all units.
+        int it = 0, vslot_prev = 0, li = 0, c0 = 0, c1 = 0, prev_c1 = 0, iu = 0;
+        bool ok = true, prev_u1 = false, prev_acc1 = false;
+        for_each_unit([&](int) -> bool {
+          if (nt == 0) return true;
+          const int qb = iu % QB;
+          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
+          const uint32_t q_buf = q_addr + 2 * qb * L::kTileBytes;
+          const int li0 = li, c00 = c0, c10 = c1;
+          for (int j = 0; j < nt && ok; ++j) {
+            const bool u0 = uses(0, j), u1 = uses(1, j);
+            if constexpr (SPARSE) {
+              if (!u0 && !u1) continue;
+            } else {  // dense: every key tile is in the ring and each tile uses a prefix
+              li = li0 + j;
+              it = 2 * li;
+              c0 = c00 + j;
+              c1 = c10 + j;
             }
-            umma_commit(&kv_empty[vslot_prev]);
+            const int kslot = it % S;
+            if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + li * 16 + 0);
+            ++it;
+            if (u0) {
+              issue_qk(0, kslot, q_buf);
+              MEA_TRACE_AT(1024 + li * 16 + 1);
+              umma_commit(&s_full[0]);
+            }
+            if (li >= 1) {  // P1.V of the previous ring step (maybe of the previous unit)
+              if (prev_u1) {
+                if (!(ok = mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status))) break;
+                MEA_TRACE_AT(1024 + li * 16 + 2);
+                tc_fence_after();
+                issue_pv(1, vslot_prev, prev_acc1);
+                umma_commit(&o_done[1]);
+              }
+              umma_commit(&kv_empty[vslot_prev]);
+            }
+            if (u1) {
+              issue_qk(1, kslot, q_buf);
+              MEA_TRACE_AT(1024 + li * 16 + 3);
+              umma_commit(&s_full[1]);
+            }
+            // This unit's Q buffer is free once its last Q.K^T MMAs have completed.
+            if (kPersist && j == nt - 1) umma_commit(&q_empty[qb]);
+            umma_commit(&kv_empty[kslot]);
+            const int vslot = it % S;
+            if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(1024 + li * 16 + 4);
+            ++it;
+            if (u0) {
+              if (!(ok = mbar_wait(&p_ready[0], c0 & 1, abort_flag, a.status))) break;
+              MEA_TRACE_AT(1024 + li * 16 + 5);
+              tc_fence_after();
+              issue_pv(0, vslot, c0 > c00);
+              MEA_TRACE_AT(1024 + li * 16 + 6);
+              umma_commit(&o_done[0]);
+              ++c0;
+            }
+            vslot_prev = vslot;
+            prev_u1 = u1;
+            prev_acc1 = c1 > c10;  // P.V accumulates after the unit's first key tile
+            prev_c1 = c1;
+            c1 += u1 ? 1 : 0;
+            ++li;
           }
-          if (u1) {
-            issue_qk(1, kslot, q_addr);
-            MEA_TRACE_AT(1024 + li * 16 + 3);
-            umma_commit(&s_full[1]);
+          if constexpr (!SPARSE) {
+            li = li0 + nt;
+            it = 2 * li;
+            c0 = c00 + nt_tile[0];
+            c1 = c10 + nt_tile[1];
           }
-          umma_commit(&kv_empty[kslot]);
-          const int vslot = it % S;
-          if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
-          MEA_TRACE_AT(1024 + li * 16 + 4);
-          ++it;
-          if (u0) {
-            if (!(ok = mbar_wait(&p_ready[0], c0 & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + li * 16 + 5);
-            tc_fence_after();
-            issue_pv(0, vslot, c0 > 0);
-            MEA_TRACE_AT(1024 + li * 16 + 6);
-            umma_commit(&o_done[0]);
-            ++c0;
-          }
-          vslot_prev = vslot;
-          prev_u1 = u1;
-          prev_c1 = c1;
-          c1 += u1 ? 1 : 0;
-          ++li;
-        }
-        if constexpr (!SPARSE) li = nt;
+          ++iu;
+          return ok;
+        });
         if (ok && li > 0) {
           if (prev_u1 && mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status)) {
             tc_fence_after();
-            issue_pv(1, vslot_prev, prev_c1 > 0);
+            issue_pv(1, vslot_prev, prev_acc1);
             umma_commit(&o_done[1]);
           }
           umma_commit(&kv_empty[vslot_prev]);
@@ -696,8 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale_log2 = fmaxf(a.scale_log2, 1e-30f);
     bool ok = true;
     int nc = 0;  // key tiles this query tile has computed, over all units (barrier phases)
-    for (int cu = blockIdx.x;; cu += gridDim.x) {
-      if (kPersist) next_unit(cu);
+    for_each_unit([&](int ku) -> bool {
       const int nbase = nc;  // nc at the unit's start
       const int ntt = nt_tile[t];
       int rr[2], pos[2];
@@ -718,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
         if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
-        if (tracer && t == 0 && j == 0 && cu == blockIdx.x) MEA_CTA_AT(1);
+        if (tracer && t == 0 && j == 0 && ku == 0) MEA_CTA_AT(1);
         // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
         // need no masking for any row of the warp take the unmasked path.
         int n0 = j * kBN, kfirst = 0;
@@ -919,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++nc;
       }
       if constexpr (!SPARSE) nc = nbase + ntt;
-      if (tracer && t == 0 && cu == blockIdx.x) MEA_CTA_AT(2);
+      if (tracer && t == 0 && ku == 0) MEA_CTA_AT(2);
 
       // ---- epilogue: out = O / l, lse = (m + log2 l) * ln 2 ---------------------
       // (Persistent instances recompute the rows here rather than keep them in
@@ -962,9 +961,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (tracer && t == 0 && cu == blockIdx.x) MEA_CTA_AT(3);
-      if (!kPersist || !ok || cu + static_cast<int>(gridDim.x) >= n_units) break;
-    }
+      if (tracer && t == 0 && ku == 0) MEA_CTA_AT(3);
+      return ok;
+    });
   }
 
   tc_fence_before();
@@ -995,10 +994,10 @@ cudaError_t sm_count(int* out) {
 
 template <int D, bool BF16, int MASK, bool ALIBI, int MODE = kModeDense>
 cudaError_t launch_t(const FwdLaunch& L, cudaStream_t stream) {
-  auto kern = fwd_kernel<D, BF16, MASK, ALIBI, MODE>;
+  constexpr auto kern = fwd_kernel<D, BF16, MASK, ALIBI, MODE>;
   constexpr bool kPersist = kPersistent<D, BF16, MASK, ALIBI, MODE>;
-  const int smem = Smem<D, kPersist ? 2 : 1>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = Smem<D, kQBuffers<D, BF16, MASK, ALIBI, MODE>>::kBytes;
+  cudaError_t e = set_smem_once<kern>(smem);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(L.args.num_mblocks) * L.args.Hq *
                          L.args.num_units;

@@ -262,3 +262,17 @@ def test_grouped_5d_layout(mea, orc, expanded):
     ro, rl = orc.attention(q5.reshape(B, M, G * H, K), k_rep, v_rep, bias=1, scale=K ** -0.5)
     assert_out_close(out.reshape(B, M, G * H, K), ro, "5-D grouped")
     assert_lse_close(lse, rl, "5-D grouped")
+
+
+def test_prepared_call_matches_plain_call(mea):
+    """A prepared mea_fwd (arguments marshalled once) gives the plain call's
+    results bit for bit, call after call."""
+    p = synth.causal_small()
+    q, k, v = p.q.to(DEV), p.k.to(DEV), p.v.to(DEV)
+    ref = mea.mea_fwd(q, k, v, bias="causal", scale=p.scale)
+    call = mea.mea_fwd(q, k, v, bias="causal", scale=p.scale, prepare=True)
+    for _ in range(3):
+        out, lse = call()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
+    assert mea.read_device_status() == 0
