@@ -194,7 +194,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nb = blockIdx.x, kvh = blockIdx.y, unit = blockIdx.z;
+  // CTA -> (key block, kv head, batch or sequence).  Under a causal mask a key
+  // block's work falls with its index (block 0 sees every query row, the last
+  // block only the last rows), so the key block varies slowest and the heaviest
+  // CTAs of the launch start first; otherwise it varies fastest, so the CTAs of
+  // one (kv head, batch) run together and share their Q / dO reads in L2.
+  int nb = blockIdx.x, kvh = blockIdx.y, unit = blockIdx.z;
+  if constexpr (MASK == 1 || MASK == 3) {
+    const int l = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int per = gridDim.y * gridDim.z;
+    nb = l / per;
+    kvh = (l - nb * per) % gridDim.y;
+    unit = (l - nb * per) / gridDim.y;
+  }
 
   int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, bidx = unit;
   if constexpr (kPacked) {

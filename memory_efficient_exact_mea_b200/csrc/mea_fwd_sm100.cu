@@ -65,7 +65,12 @@ struct Smem {
   static constexpr int kNumBars = 2 * QB + 2 * kSlots + 2 + 2 + 2 + 1 + 2;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kBytes = kAbort + 4 + 1024;  // + slack to align the base to 1024
+  // Packed causal batches: sequences by decreasing length, and where each query
+  // block level starts in the unit ranks (see fwd_kernel).
+  static constexpr int kMaxSeqs = 256, kMaxLevels = 64;
+  static constexpr int kSeqOrder = kAbort + 4;                  // int16[kMaxSeqs]
+  static constexpr int kLevelStart = kSeqOrder + 2 * kMaxSeqs;  // int32[kMaxLevels + 1]
+  static constexpr int kBytes = kLevelStart + 4 * (kMaxLevels + 1) + 1024;  // + base alignment
 };
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -200,7 +205,76 @@ __global__ void __launch_bounds__(kThreads, 1)
   // a causal mask a unit's work grows with its query block, so the ranks go by
   // query block, last (longest rows) first, with the heads fastest: the longest
   // units of the whole launch start first.
-  const int n_ranks = a.num_mblocks * a.Hq * a.num_units;
+  // Packed batches under a causal mask: most units of the rank space above
+  // would be empty (a short sequence has no late query blocks), and a fixed
+  // order that skips empty ranks spreads the real ones unevenly.  There the
+  // CTA first sorts the sequences by decreasing length (up to kMaxSeqs of them)
+  // and ranks only units that exist: level l (query block num_mblocks - 1 - l)
+  // holds the sequences longer than that block's first row, longest first,
+  // heads fastest.  A sequence whose offsets are invalid is recorded in the
+  // status word and gets no units.
+  int16_t* seq_order = reinterpret_cast<int16_t*>(smem + L::kSeqOrder);
+  int* level_start = reinterpret_cast<int*>(smem + L::kLevelStart);
+  constexpr bool kCompactable = kPacked && kCausal;
+  const bool compact =
+      kCompactable && a.num_units <= L::kMaxSeqs && a.num_mblocks <= L::kMaxLevels;
+  // Chunked prefill: a unit's work is its sequence's cached rows plus the new
+  // ones, which differ widely between sequences, so the sequences are ranked by
+  // that (decreasing, up to kMaxSeqs of them) and the units of the longest go
+  // first; within a sequence as elsewhere (causal: last query block first).
+  const bool by_keys = kCache && a.num_units <= L::kMaxSeqs;
+  if constexpr (kCache) {
+    if (by_keys) {
+      auto keys_of = [&](int s) -> int { return a.cache_len[s] + (a.q_lens ? a.q_lens[s] : a.M); };
+      for (int i = threadIdx.x; i < a.num_units; i += kThreads) {
+        const int ki = keys_of(i);
+        int pos = 0;
+        for (int j = 0; j < a.num_units; ++j) {
+          const int kj = keys_of(j);
+          pos += (kj > ki) || (kj == ki && j < i);
+        }
+        seq_order[pos] = static_cast<int16_t>(i);
+      }
+      __syncthreads();
+    }
+  }
+  if constexpr (kCompactable) {
+    if (compact) {
+      auto rows_of = [&](int s) -> int {  // query rows of sequence s; 0 if its offsets are invalid
+        const int qs = a.seqstart_q[s], ql = a.seqstart_q[s + 1] - qs;
+        const int ks = a.seqstart_k[s], kl = a.seqstart_k[s + 1] - ks;
+        const bool bad = ql < 0 || kl < 0 || qs < 0 || ks < 0 || qs + ql > a.M ||
+                         ks + kl > a.N || ql > a.num_mblocks * kFwdRowsPerCta;
+        return bad ? -1 : ql;
+      };
+      for (int i = threadIdx.x; i < a.num_units; i += kThreads) {
+        const int li = rows_of(i);
+        if (li < 0) record_error(a.status, kErrInvalidArg);
+        int pos = 0;
+        for (int j = 0; j < a.num_units; ++j) {
+          const int lj = rows_of(j);
+          pos += (lj > li) || (lj == li && j < i);
+        }
+        seq_order[pos] = static_cast<int16_t>(i);
+      }
+      for (int l = threadIdx.x; l < a.num_mblocks; l += kThreads) {
+        const int first_row = (a.num_mblocks - 1 - l) * kFwdRowsPerCta;
+        int c = 0;
+        for (int j = 0; j < a.num_units; ++j) c += rows_of(j) > first_row;
+        level_start[l + 1] = c * a.Hq;  // units of level l, summed below
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        level_start[0] = 0;
+        for (int l = 0; l < a.num_mblocks; ++l) level_start[l + 1] += level_start[l];
+      }
+      __syncthreads();
+    }
+  }
+  int n_ranks = a.num_mblocks * a.Hq * a.num_units;
+  if constexpr (kCompactable) {
+    if (compact) n_ranks = level_start[a.num_mblocks];
+  }
   int mb = 0, h = 0, unit = 0, kvh = 0, bidx = 0, m_base = 0;
   int q0 = 0, q_len = a.M, k0 = 0, k_len = a.N, off = 0;
   int past = 0;  // cache mode: rows cached before this chunk
@@ -213,7 +287,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   // offsets are invalid (the status word records it; nothing to do), 1 if the
   // unit has no query rows, 2 if it has rows to compute.
   auto set_unit = [&](int rank) -> int {
-    if constexpr (kCausal) {
+    if (kCompactable && compact) {
+      int l = 0;
+      while (rank >= level_start[l + 1]) ++l;
+      const int i = rank - level_start[l];
+      h = i % a.Hq;
+      unit = seq_order[i / a.Hq];
+      mb = a.num_mblocks - 1 - l;
+    } else if (kCache && by_keys) {
+      const int per = a.Hq * a.num_mblocks;
+      const int pos = rank / per;
+      const int rem = rank - pos * per;
+      unit = seq_order[pos];
+      if (kCausal) {
+        h = rem % a.Hq;
+        mb = a.num_mblocks - 1 - rem / a.Hq;
+      } else {
+        mb = rem % a.num_mblocks;
+        h = rem / a.num_mblocks;
+      }
+    } else if constexpr (kCausal) {
       const int per = a.Hq * a.num_units;
       const int level = rank / per;
       const int rem = rank - level * per;

@@ -1,12 +1,17 @@
 """Parity of the backward kernels (mea_bwd, through the C ABI) with the fp64
 oracle's gradients on the same seeded inputs and upstream gradient.
 
-Tolerance (derived, gradients only): the GPU forms D_i = <dO_i, O_i> from the
-forward's fp16/bf16 output O, whose rounding (relative 2^-11 / 2^-8) enters every
-dS_ij = p_ij (dP_ij - D_i) of the row; P and dS are carried with >= 11 (fp16) or
-~16 (bf16 hi+lo) significant bits and accumulated in fp32.  Elementwise:
+Tolerance (gradients only).  Elementwise, per tensor (dq, dk, dv):
     |g - ref| <= rtol * |ref| + atol * max|ref|,  rtol = 2e-2,
-    atol = 4e-3 (fp16) / 1e-2 (bf16)  (per tensor: dq, dk, dv)."""
+    atol = 1e-3 (fp16) / 8e-3 (bf16).
+Where the error comes from: the GPU forms D_i = <dO_i, O_i> from the forward's
+16-bit output O, and P^T and dS^T enter the dV, dK and dQ products as single
+16-bit values (relative rounding 2^-12 for fp16, 2^-9 for bf16), accumulated in
+fp32; every gradient element sums many such terms, whose rounding errors mostly
+cancel.  The largest atol any case here needed, measured on the GPU against the
+oracle (every case of this file, the rescale file's backward and two groups of
+each full-size workload), was 2.7e-4 (fp16) and 4.5e-3 (bf16, keys ramped 1 ->
+16); the bounds above keep a margin of about 4x and 1.8x over those."""
 import numpy as np
 import pytest
 import torch
@@ -30,7 +35,7 @@ def _assert_grad(g, ref, dtype, what):
     g, r = to_np(g), to_np(ref)
     assert np.isfinite(g).all(), f"{what}: non-finite"
     scale = np.abs(r).max() + 1e-30
-    atol = (4e-3 if dtype == "f16" else 1e-2) * scale
+    atol = (1e-3 if dtype == "f16" else 8e-3) * scale
     err = np.abs(g - r)
     bad = err > atol + 2e-2 * np.abs(r)
     assert not bad.any(), (f"{what}: {bad.sum()}/{bad.size} out of tolerance, max err "

@@ -276,3 +276,15 @@ def test_prepared_call_matches_plain_call(mea):
         torch.cuda.synchronize()
         assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
     assert mea.read_device_status() == 0
+
+
+@pytest.mark.parametrize("n_seqs", [200, 300])
+def test_varlen_many_sequences(mea, orc, n_seqs):
+    """Packed causal batches with many sequences (lengths 0 .. 700, a few at the
+    maximum): up to 256 sequences the CTAs rank only the units that exist
+    (sequences sorted by length), beyond that every (block, head, sequence)
+    rank, skipping empty ones.  Every element against the oracle."""
+    lens = [int(x) for x in synth.lengths(n_seqs, 0, 700, synth.generator(95 + n_seqs))]
+    lens[3] = lens[n_seqs // 2] = 700
+    p = synth.make_varlen(f"varlen_{n_seqs}", lens, 4, 2, 64, "f16", True, seed=96)
+    _check_full(mea, orc, p)
