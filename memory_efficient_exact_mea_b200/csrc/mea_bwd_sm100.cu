@@ -103,22 +103,25 @@ struct BwdCfg {
   static constexpr int kKVTile = kChunksD * kKVChunk;
   static constexpr int kQTile = kChunksD * kQChunk;
   static constexpr int kDSTile = (BM / 64) * kKVChunk;  // dS^T: 128 keys x BM queries
-  static constexpr int kStages = 3;                   // Q / dO stages
+  // Q / dO stages: three at K = 128; two at K = 64, where a third does not fit
+  // beside the dQ staging buffer.
+  static constexpr int kStages = (D == 128) ? 3 : 2;
   static constexpr int kStage = 2 * kQTile;           // Q then dO
   static constexpr int kDQSBox = BM * 128;            // dQ staging: D/32 boxes of BM x 128 B
-  static_assert((D / 32) * kDQSBox == kStage, "dQ staging fills one Q/dO stage");
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kK = 0;
   static constexpr int kV = kKVTile;
   static constexpr int kQD = 2 * kKVTile;              // stage i: Q at kQD + i*kStage, dO after it
   static constexpr int kDS = kQD + kStages * kStage;   // two buffers (step parity)
-  static constexpr int kLse = kDS + 2 * kDSTile;      // [stage][BM] -lse * log2(e) (-inf: no weight)
+  static constexpr int kDQS = kDS + 2 * kDSTile;       // dQ of one step, fp32, for the reductions
+  static constexpr int kLse = kDQS + (D / 32) * kDQSBox;  // [stage][BM] -lse * log2(e) (-inf: no weight)
   static constexpr int kDelta = kLse + kStages * BM * 4;  // [stage][BM] -D
   static constexpr int kBar = kDelta + kStages * BM * 4;
   static constexpr int kNumBars = 14;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4 + 1024;
+  static_assert(kBytes <= 227 * 1024, "shared memory");
   // tensor memory columns (every region starts on a multiple of 64):
   //   K = 64:  S^T 0 | dP^T 128 | P^T 256 (64) | dQ 320 | dV 384 | dK 448
   //   K = 128: S^T 0 | dP^T 64 | dQ 128 | dV 192 | dK 320 | P^T 448 (32)
@@ -130,35 +133,50 @@ struct BwdCfg {
   static_assert(kColDK + D <= kTmemCols && kColP + BM / 2 <= kTmemCols, "tensor memory layout");
 };
 
-// One warp per (row, query head): D = <dout, out>, and zero the dq accumulator row.
+// D = <dout, out> per (row, query head), and the row's dq accumulator zeroed.
+// A row is K / 8 lanes of 16-byte loads (8 at K = 64, 16 at K = 128), so a warp
+// covers 4 or 2 rows with fully used 16-byte accesses.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  constexpr int kLanes = D / 8;  // lanes per row, 8 elements each
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = t / kLanes;
+  const int part = static_cast<int>(t % kLanes);
   const long long rows = static_cast<long long>(a.B) * a.M * a.Hq;
-  if (row >= rows) return;
-  const long long b = row / (static_cast<long long>(a.M) * a.Hq);
-  const long long i = (row / a.Hq) % a.M;
-  const long long h = row % a.Hq;
-  const uint16_t* o = static_cast<const uint16_t*>(a.out) + row * D;
-  const uint16_t* g = static_cast<const uint16_t*>(a.dout) + row * D;
+  const bool live = row < rows;
   float s = 0.f;
+  if (live) {
+    const uint4 o = reinterpret_cast<const uint4*>(a.out)[row * kLanes + part];
+    const uint4 g = reinterpret_cast<const uint4*>(a.dout)[row * kLanes + part];
+    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-  for (int d = lane; d < D; d += 32) s = fmaf(to_f<BF16>(o[d]), to_f<BF16>(g[d]), s);
+    for (int w = 0; w < 4; ++w) {
+      s = fmaf(to_f<BF16>(static_cast<uint16_t>(ow[w] & 0xffffu)),
+               to_f<BF16>(static_cast<uint16_t>(gw[w] & 0xffffu)), s);
+      s = fmaf(to_f<BF16>(static_cast<uint16_t>(ow[w] >> 16)),
+               to_f<BF16>(static_cast<uint16_t>(gw[w] >> 16)), s);
+    }
+    float4* acc = reinterpret_cast<float4*>(a.dq_acc + row * D + part * 8);
+    acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) a.delta[(b * a.Hq + h) * a.M + i] = s;
-#pragma unroll
-  for (int d = lane; d < D; d += 32) a.dq_acc[row * D + d] = 0.f;
+  for (int off = kLanes / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (live && part == 0) {
+    const long long b = row / (static_cast<long long>(a.M) * a.Hq);
+    const long long i = (row / a.Hq) % a.M;
+    const long long h = row % a.Hq;
+    a.delta[(b * a.Hq + h) * a.M + i] = s;
+  }
 }
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_dq_out_kernel(const BwdArgs a) {
-  const long long n = static_cast<long long>(a.B) * a.M * a.Hq * D / 2;
+  const long long n = static_cast<long long>(a.B) * a.M * a.Hq * D / 4;  // 4 elements each
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float2 v = reinterpret_cast<const float2*>(a.dq_acc)[e];
-    reinterpret_cast<uint32_t*>(a.dq)[e] = pack2<BF16>(v.x, v.y);
+    const float4 v = reinterpret_cast<const float4*>(a.dq_acc)[e];
+    reinterpret_cast<uint2*>(a.dq)[e] = make_uint2(pack2<BF16>(v.x, v.y), pack2<BF16>(v.z, v.w));
   }
 }
 
@@ -179,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NS = C::kStages;
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;        // [NS] Q, dO (+ lse, D) of a step landed
-  uint64_t* q_empty = bars + 1 + NS;  // [NS] the stage is free again (its dQ reductions read it)
+  uint64_t* q_empty = bars + 1 + NS;  // [NS] the stage is free again (its MMAs completed)
   uint64_t* s_full = bars + 1 + 2 * NS;   // S^T, dP^T of the step are in TMEM
   uint64_t* s_free = s_full + 1;      // S^T, dP^T read out of TMEM (256 arrivals)
   uint64_t* p_ready = s_full + 2;     // P^T in TMEM and dS^T in shared memory (256 arrivals)
@@ -392,6 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ss(tDK, sdesc_sw128(sDS + (kk >> 2) * C::kKVChunk + (kk & 3) * 32, 16, 1024),
                   sdesc_sw128(sQ + kk * 2048, C::kQChunk, 1024), idesc_g,
                   (s > 0 || kk > 0) ? 1u : 0u);
+        // No later MMA reads this step's Q / dO stage: the loader may refill it
+        // once these have completed.
+        umma_commit(&q_empty[slot]);
         // dQ: both operands M/N-contiguous views of row-major 128-key tiles, 16 keys
         // (2048 bytes) per step.  K = 128: dQ^T = K^T dS^T; K = 64: dQ = dS K.
         BWD_TRACE(s, 4);
@@ -585,8 +606,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait_warp(dq_full, s & 1, abort_flag, a.status))) break;
       if (leader) BWD_TRACE(s, 16);
       tc_fence_after();
-      // Stage dQ in this step's Q / dO stage: every MMA reading it has completed.
-      uint8_t* stage = smem + C::kQD + (s % NS) * C::kStage;
+      // Stage dQ in the staging buffer, once the previous step's reductions have
+      // read it (the leader waits for them, then joins this barrier).
+      uint8_t* stage = smem + C::kDQS;
+      if (s > 0) named_sync(2, 128);
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
         uint32_t v[32];
@@ -627,8 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < D / 32; ++b)
           tma_reduce_add_4d(&tmDQ, stage + b * C::kDQSBox, 32 * b, h, q0 + m0, bidx);
         bulk_commit();
-        bulk_wait_read();
-        mbar_arrive(&q_empty[s % NS]);  // the loader may refill the stage
+        bulk_wait_read();  // the staging buffer may be written again
       }
     }
     if (leader) bulk_wait_all();
@@ -661,7 +683,8 @@ cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream, int stages) {
   if (rows <= 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   if (stages & 1) {
-    bwd_prep_kernel<D, BF16><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(a);
+    bwd_prep_kernel<D, BF16>
+      <<<static_cast<unsigned>((rows * (D / 8) + 255) / 256), 256, 0, stream>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -680,8 +703,8 @@ cudaError_t launch_all(const BwdLaunch& L, cudaStream_t stream, int stages) {
     if (e != cudaSuccess) return e;
   }
   if (!(stages & 4)) return cudaSuccess;
-  const long long pairs = rows * D / 2;
-  const long long blocks = std::min((pairs + 255) / 256, 148LL * 16);
+  const long long quads = rows * D / 4;
+  const long long blocks = std::min((quads + 255) / 256, 148LL * 16);
   bwd_dq_out_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
