@@ -46,7 +46,7 @@ constexpr int kBN = 128;        // keys per tile
 constexpr int kThreads = 608;
 constexpr int kMmaWarp = 16;   // + tile: warps 16 and 17 each issue one query tile's MMAs
 constexpr int kTmaWarp = 18;
-constexpr int kSoftmaxThreadsPerTile = 256;  // four threads per row
+constexpr int kSoftmaxWarpsPerTile = 8;  // four threads per row, 16 rows per warp
 constexpr uint32_t kTmemCols = 512;
 constexpr float kTau = 8.0f;    // keep a stale row max while the new one exceeds it by < 2^8
 constexpr float kLog2e = 1.4426950408889634f;
@@ -62,7 +62,7 @@ struct Smem {
   static constexpr int kQ = 0;
   static constexpr int kKV = QB * 2 * kTileBytes;
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  static constexpr int kNumBars = 2 * QB + 2 * kSlots + 2 + 2 + 2 + 1 + 2;
+  static constexpr int kNumBars = 2 * QB + 2 * kSlots + 2 + 8 + 2 + 1 + 2;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   // Packed causal batches: sequences by decreasing length, and where each query
@@ -85,11 +85,15 @@ __device__ __forceinline__ int opaque(int x) {
 
 // Pipeline timeline for performance work: built only with -DMEA_TRACE, it
 // records clock64() at each pipeline event of the first kTraceCtas CTAs.
-// Slots per CTA: softmax tile t, key tile j, event e -> t*512 + j*16 + e;
-// MMA thread, key tile j, event e -> 1024 + j*16 + e (j < 32).
+// Slots per CTA (step counters modulo 256): softmax tile t, its step n, event e
+// -> t*4096 + n*16 + e; MMA thread, ring step l, event e -> 8192 + l*16 + e (one
+// issuing thread) or 8192 + t*2048 + l*8 + e (one per tile); unit k (modulo 64),
+// softmax tile t -> 12288 + k*4 + 2t (start), + 1 (epilogue done); TMA ring copy
+// i (modulo 512) issued -> 12544 + 2i; Q load of unit k (modulo 64) -> 13568 + k;
+// softmax warp w, step n: P published -> 13632 + w*256 + n.
 #ifdef MEA_TRACE
 constexpr int kTraceCtas = 4;
-constexpr int kTraceSlots = 1536;
+constexpr int kTraceSlots = 17728;
 __device__ long long g_trace[kTraceCtas * kTraceSlots];
 #define MEA_TRACE_AT(slot)                                                         \
   do {                                                                             \
@@ -186,8 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* kv_full = bars + 2 * QB;
   uint64_t* kv_empty = bars + 2 * QB + S;
   uint64_t* s_full = bars + 2 * QB + 2 * S;
+  // p_ready[4t + C]: P of tile t published; with P written over S, C counts its
+  // 32-key chunks (the P.V MMAs of a chunk go out once it is published); the
+  // separate-P layout publishes the whole tile on p_ready[4t].
   uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 2;
+  uint64_t* o_done = p_ready + 8;
   uint64_t* mma_done = o_done + 2;
   uint64_t* s_free = mma_done + 1;    // S_t read out by the softmax (separate-P layout)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
@@ -467,11 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_ready[t], kSoftmaxThreadsPerTile);
+      for (int c = 0; c < 4; ++c) mbar_init(&p_ready[4 * t + c], kSoftmaxWarpsPerTile);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(mma_done, kSepP ? 2 : 1);
-    for (int t = 0; t < 2; ++t) mbar_init(&s_free[t], kSoftmaxThreadsPerTile);
+    for (int t = 0; t < 2; ++t) mbar_init(&s_free[t], kSoftmaxWarpsPerTile);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -510,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sQ + (2 * qb + t) * L::kTileBytes + c * L::kChunkBytes, &tmQ, &q_full[qb],
                         c * 64, h, q0 + m_base + t * kBM, bidx);
+        MEA_TRACE_AT(13568 + (iu & 63));
         ++iu;
         for (int j = 0; j < nt; ++j) {
           if constexpr (SPARSE) {
@@ -525,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < L::kChunks; ++c)
               tma_load_4d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, map, &kv_full[slot],
                           c * 64, kvh, kt.row, bidx);
+            MEA_TRACE_AT(12544 + (it & 511) * 2);
           }
           if (*abort_flag) return false;
         }
@@ -538,8 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
     // ===================== MMA issuers, one per query tile ====================
+    // The whole warp runs the issuing loop (all values warp-uniform); elect.sync
+    // picks the lane that issues each MMA and commit.
     const int tile = warp - kMmaWarp;
-    if (lane == 0) {
+    {
       const uint32_t idesc_qk = idesc_f16(BF16, kBM, kBN, false);
       const uint32_t idesc_pv = idesc_f16(BF16, kBM, D, true);
       const uint32_t q_addr = smem_u32(sQ);
@@ -553,30 +564,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t o = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-          umma_ss(d, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(kb + o, 16, 1024), idesc_qk,
+          umma_ss_warp(d, sdesc_sw128(qa + o, 16, 1024), sdesc_sw128(kb + o, 16, 1024), idesc_qk,
                   kk > 0);
         }
       };
-      // O_t (+)= P_t V: P from TMEM (2 elements per column; keys 32c..32c+31 in
-      // columns 32c..32c+15), V N-major with its 64-column chunks L::kChunkBytes
-      // apart; step k covers 16 keys = 2048 bytes of V.  With the bf16 split the
-      // low part P_lo (16 columns further) goes through the same V descriptors.
-      // Separate-P layout: keys 2c, 2c+1 in column c of P_t.
+      // O_t (+)= P_t V with P read from TMEM (two 16-bit elements per column) and V
+      // N-major, its 64-column chunks L::kChunkBytes apart; step k covers 16 keys =
+      // 2048 bytes of V.  Separate-P layout: keys 2c, 2c+1 in column c of P_t.
       auto issue_pv = [&](int t, int slot, bool accumulate) {
         const uint32_t d = tmem_base + kColO + t * D;
-        const uint32_t p = tmem_base + kColP + t * (kSepP ? kBN / 2 : kBN);
+        const uint32_t p = tmem_base + kColP + t * (kBN / 2);
         const uint32_t vb = kv_addr + slot * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts(d, kSepP ? p + kk * 8 : p + (kk >> 1) * 32 + (kk & 1) * 8,
-                  sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
+          umma_ts_warp(d, p + kk * 8, sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
                   (accumulate || kk > 0) ? 1u : 0u);
-        if constexpr (kSplitP) {
+      };
+      // P over S: keys 32c..32c+31 in columns 32c..32c+15 (bf16: P_hi there and
+      // P_lo = P - P_hi in the 16 columns after, through the same V descriptors).
+      // The MMAs of each 32-key chunk go out as soon as the softmax has published
+      // that chunk, so the contraction runs alongside the rest of the tile's softmax.
+      auto pv_chunks = [&](int t, int slot, bool accumulate, uint32_t parity) -> bool {
+        const uint32_t d = tmem_base + kColO + t * D;
+        const uint32_t p = tmem_base + kColP + t * kBN;
+        const uint32_t vb = kv_addr + slot * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts(d, p + (kk >> 1) * 32 + 16 + (kk & 1) * 8,
-                    sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv, 1u);
+        for (int c = 0; c < 4; ++c) {
+          if (!mbar_wait_warp(&p_ready[4 * t + c], parity, abort_flag, a.status)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int part = 0; part < (kSplitP ? 2 : 1); ++part)
+#pragma unroll
+            for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
+              umma_ts_warp(d, p + c * 32 + part * 16 + (kk & 1) * 8,
+                      sdesc_sw128(vb + kk * 2048, L::kChunkBytes, 1024), idesc_pv,
+                      (accumulate || kk > 0 || part > 0) ? 1u : 0u);
         }
+        return true;
       };
 
       // Ring index 2j holds K_j, 2j+1 holds V_j; each slot is released when both
@@ -590,17 +614,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = tile;
       auto pv_step = [&](int lv, bool used, int cu, bool acc) -> bool {
         const int vs = (2 * lv + 1) % S;
-        if (!mbar_wait(&kv_full[vs], ((2 * lv + 1) / S) & 1, abort_flag, a.status)) return false;
-        MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 2);
+        if (!mbar_wait_warp(&kv_full[vs], ((2 * lv + 1) / S) & 1, abort_flag, a.status)) return false;
+        MEA_TRACE_AT(8192 + t * 2048 + (lv & 255) * 8 + 2);
         if (used) {
-          if (!mbar_wait(&p_ready[t], cu & 1, abort_flag, a.status)) return false;
-          MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 3);
+          if (!mbar_wait_warp(&p_ready[4 * t], cu & 1, abort_flag, a.status)) return false;
+          MEA_TRACE_AT(8192 + t * 2048 + (lv & 255) * 8 + 3);
           tc_fence_after();
           issue_pv(t, vs, acc);
-          umma_commit(&o_done[t]);
-          MEA_TRACE_AT(1024 + t * 256 + lv * 8 + 4);
+          umma_commit_warp(&o_done[t]);
+          MEA_TRACE_AT(8192 + t * 2048 + (lv & 255) * 8 + 4);
         }
-        umma_commit(&kv_empty[vs]);
+        umma_commit_warp(&kv_empty[vs]);
         return true;
       };
       // Separate-P layout: one thread per query tile.  P.V stays one step behind
@@ -614,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for_each_unit([&](int) -> bool {
           if (nt == 0) return true;
           const int qb = iu % QB;
-          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
+          if (!(ok = mbar_wait_warp(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
           const uint32_t q_buf = q_addr + 2 * qb * L::kTileBytes;
           const int li0 = li, c0 = c;
           for (int j = 0; j < nt && ok; ++j) {
@@ -626,18 +650,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               c = c0 + j;
             }
             const int ks = (2 * li) % S;
-            if (!(ok = mbar_wait(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + t * 256 + li * 8 + 0);
+            if (!(ok = mbar_wait_warp(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(8192 + t * 2048 + (li & 255) * 8 + 0);
             if (used) {
               if (c > 0) {  // the softmax has read the previous S_t out of TMEM
-                if (!(ok = mbar_wait(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
+                if (!(ok = mbar_wait_warp(&s_free[t], (c - 1) & 1, abort_flag, a.status))) break;
                 tc_fence_after();
               }
               issue_qk(t, ks, q_buf);
-              umma_commit(&s_full[t]);
-              MEA_TRACE_AT(1024 + t * 256 + li * 8 + 1);
+              umma_commit_warp(&s_full[t]);
+              MEA_TRACE_AT(8192 + t * 2048 + (li & 255) * 8 + 1);
             }
-            umma_commit(&kv_empty[ks]);
+            umma_commit_warp(&kv_empty[ks]);
             if (li >= 1) ok = pv_step(li - 1, prev_used, prev_c, prev_acc);
             prev_used = used;
             prev_acc = c > c0;  // P.V accumulates after the unit's first key tile
@@ -650,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             c = c0 + nt_tile[t];
           }
           // This unit's Q buffer is free once its Q.K^T MMAs have completed.
-          if constexpr (kPersist) umma_commit(&q_empty[qb]);
+          if constexpr (kPersist) umma_commit_warp(&q_empty[qb]);
           ++iu;
           return ok;
         });
@@ -671,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for_each_unit([&](int) -> bool {
           if (nt == 0) return true;
           const int qb = iu % QB;
-          if (!(ok = mbar_wait(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
+          if (!(ok = mbar_wait_warp(&q_full[qb], (iu / QB) & 1, abort_flag, a.status))) return false;
           const uint32_t q_buf = q_addr + 2 * qb * L::kTileBytes;
           const int li0 = li, c00 = c0, c10 = c1;
           for (int j = 0; j < nt && ok; ++j) {
@@ -685,43 +709,39 @@ __global__ void __launch_bounds__(kThreads, 1)
               c1 = c10 + j;
             }
             const int kslot = it % S;
-            if (!(ok = mbar_wait(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + li * 16 + 0);
+            if (!(ok = mbar_wait_warp(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(8192 + (li & 255) * 16 + 0);
             ++it;
             if (u0) {
               issue_qk(0, kslot, q_buf);
-              MEA_TRACE_AT(1024 + li * 16 + 1);
-              umma_commit(&s_full[0]);
+              MEA_TRACE_AT(8192 + (li & 255) * 16 + 1);
+              umma_commit_warp(&s_full[0]);
             }
             if (li >= 1) {  // P1.V of the previous ring step (maybe of the previous unit)
               if (prev_u1) {
-                if (!(ok = mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status))) break;
-                MEA_TRACE_AT(1024 + li * 16 + 2);
-                tc_fence_after();
-                issue_pv(1, vslot_prev, prev_acc1);
-                umma_commit(&o_done[1]);
+                if (!(ok = pv_chunks(1, vslot_prev, prev_acc1, prev_c1 & 1))) break;
+                MEA_TRACE_AT(8192 + (li & 255) * 16 + 2);
+                umma_commit_warp(&o_done[1]);
               }
-              umma_commit(&kv_empty[vslot_prev]);
+              umma_commit_warp(&kv_empty[vslot_prev]);
             }
             if (u1) {
               issue_qk(1, kslot, q_buf);
-              MEA_TRACE_AT(1024 + li * 16 + 3);
-              umma_commit(&s_full[1]);
+              MEA_TRACE_AT(8192 + (li & 255) * 16 + 3);
+              umma_commit_warp(&s_full[1]);
             }
             // This unit's Q buffer is free once its last Q.K^T MMAs have completed.
-            if (kPersist && j == nt - 1) umma_commit(&q_empty[qb]);
-            umma_commit(&kv_empty[kslot]);
+            if (kPersist && j == nt - 1) umma_commit_warp(&q_empty[qb]);
+            umma_commit_warp(&kv_empty[kslot]);
             const int vslot = it % S;
-            if (!(ok = mbar_wait(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
-            MEA_TRACE_AT(1024 + li * 16 + 4);
+            if (!(ok = mbar_wait_warp(&kv_full[vslot], (it / S) & 1, abort_flag, a.status))) break;
+            MEA_TRACE_AT(8192 + (li & 255) * 16 + 4);
             ++it;
             if (u0) {
-              if (!(ok = mbar_wait(&p_ready[0], c0 & 1, abort_flag, a.status))) break;
-              MEA_TRACE_AT(1024 + li * 16 + 5);
-              tc_fence_after();
-              issue_pv(0, vslot, c0 > c00);
-              MEA_TRACE_AT(1024 + li * 16 + 6);
-              umma_commit(&o_done[0]);
+              MEA_TRACE_AT(8192 + (li & 255) * 16 + 5);
+              if (!(ok = pv_chunks(0, vslot, c0 > c00, c0 & 1))) break;
+              MEA_TRACE_AT(8192 + (li & 255) * 16 + 6);
+              umma_commit_warp(&o_done[0]);
               ++c0;
             }
             vslot_prev = vslot;
@@ -741,17 +761,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           return ok;
         });
         if (ok && li > 0) {
-          if (prev_u1 && mbar_wait(&p_ready[1], prev_c1 & 1, abort_flag, a.status)) {
-            tc_fence_after();
-            issue_pv(1, vslot_prev, prev_acc1);
-            umma_commit(&o_done[1]);
-          }
-          umma_commit(&kv_empty[vslot_prev]);
+          if (prev_u1 && pv_chunks(1, vslot_prev, prev_acc1, prev_c1 & 1)) umma_commit_warp(&o_done[1]);
+          umma_commit_warp(&kv_empty[vslot_prev]);
         }
       }
       // Every MMA issued above has completed once this barrier flips.
       if (kSepP || tile == 0) {
-        umma_commit(mma_done);
+        umma_commit_warp(mma_done);
         mbar_wait_drain(mma_done, 0, a.status);
       }
     }
@@ -784,6 +800,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       else tmem_st16x256_x16(o_addr, o);
     };
     const bool tracer = wt == 0 && lane == 0;
+    // One arrival per warp on the tile's barriers (counts kSoftmaxWarpsPerTile):
+    // each thread has fenced its tensor-memory accesses (tcgen05.fence::
+    // before_thread_sync) before the warp synchronises and one lane arrives.
+    auto warp_arrive = [](uint64_t* bar) { mbar_arrive_warp(bar); };
     // A zero scale is taken as 1e-30 (the same softmax to fp32 precision for any
     // finite score), so that -inf * scale stays -inf for hidden keys.
     const float scale_log2 = fmaxf(a.scale_log2, 1e-30f);
@@ -791,6 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nc = 0;  // key tiles this query tile has computed, over all units (barrier phases)
     for_each_unit([&](int ku) -> bool {
       const int nbase = nc;  // nc at the unit's start
+      if (tracer) MEA_TRACE_AT(12288 + (ku & 63) * 4 + 2 * t);
       const int ntt = nt_tile[t];
       int rr[2], pos[2];
 #pragma unroll
@@ -809,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           nc = nbase + j;
         }
         if (!(ok = mbar_wait_warp(&s_full[t], nc & 1, abort_flag, a.status))) break;
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 0);
+        if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 0);
         if (tracer && t == 0 && j == 0 && ku == 0) MEA_CTA_AT(1);
         // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
         // need no masking for any row of the warp take the unmasked path.
@@ -840,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16x256_x16_wait(s_addr, sr);
           if constexpr (kSepP) {
             tc_fence_before();
-            mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
+            warp_arrive(&s_free[t]);  // S_t may now be overwritten by the next Q.K^T
           }
 
           // ---- pass 1: row maxima (log2 units) --------------------------------------
@@ -916,7 +937,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_ref[e] = m_use;
             nsub[e] = (m_use == neg_inf()) ? 0.f : -m_use;
           }
-          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 1);
+          if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 1);
+          // The warp's output rows need a rescale (not at a unit's first key tile,
+          // whose P.V overwrites O).  Decided here with P over S, whose chunks are
+          // published during pass 2 unless the warp rescales.
+          auto need_rescale = [&] {
+            return nc > nbase && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f);
+          };
+          [[maybe_unused]] bool resc = false;
+          if constexpr (!kSepP) resc = need_rescale();
 
           // ---- pass 2: P = 2^(logit - m), partial row sums, 16-bit pairs ------------
           // Hidden logits are -inf by now (pass 1), so one mask-free copy serves every tile.
@@ -940,7 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const f2 p = p_pair(k, e);
                   pk[2 * k + e] = pack2<BF16>(p.x, p.y);
                 }
-              if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+              if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 2);
               // P_t is still being read by P.V of the previous key tile.
               if (nc > 0 && !mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status))
                 return false;
@@ -949,7 +978,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               // P over S, one 32-key chunk C (k = 4C .. 4C + 3) at a time: the hi pairs
               // are repetitions 0..3 of a 16x128b store at the chunk's column, bf16's
-              // lo pairs repetitions 4..7.
+              // lo pairs repetitions 4..7.  Without a rescale, chunk C - 1 is published
+              // once chunk C is computed (its store has landed by then); a warp that
+              // rescales publishes every chunk after the rescale below.
 #pragma unroll
               for (int C = 0; C < 4; ++C) {
                 uint32_t pc[kSplitP ? 16 : 8];
@@ -966,21 +997,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                       pc[8 + 2 * kk + e] = pack2<BF16>(res.x, res.y);
                     }
                   }
+                if (C > 0 && !resc) {
+                  tmem_st_wait();
+                  tc_fence_before();
+                  warp_arrive(&p_ready[4 * t + C - 1]);
+                }
                 if constexpr (kSplitP) tmem_st16x128_x8(p_addr + 32 * C, pc);
                 else tmem_st16x128_x4(p_addr + 32 * C, pc);
               }
-              if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 2);
+              if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 2);
             }
             return true;
           };
           if (!pass2()) return false;
 #pragma unroll
           for (int e = 0; e < 2; ++e) l_sum[e] = l_sum[e] * alpha[e] + (ps[e].x + ps[e].y);
-          if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 3);
+          if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 3);
           // Rescale the output rows whose reference max moved (after the previous
           // P.V has written O).
-          if (nc > nbase && __any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
-            if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 6);
+          if constexpr (kSepP) resc = need_rescale();
+          if (resc) {
+            if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 6);
             if constexpr (!kSepP) {
               if (!mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status)) return false;
               tc_fence_after();
@@ -996,6 +1033,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                   o[4 * k + 2 * e + c] = __float_as_uint(__uint_as_float(o[4 * k + 2 * e + c]) * alpha[e]);
             st_o(o);
           }
+          if constexpr (!kSepP) {  // publish what is left of P (the chunks above)
+            tmem_st_wait();
+            tc_fence_before();
+            if (resc) {
+#pragma unroll
+              for (int c = 0; c < 3; ++c) warp_arrive(&p_ready[4 * t + c]);
+            }
+            warp_arrive(&p_ready[4 * t + 3]);
+          }
           return true;
         };
         // Two specialised copies where that compiles best (no register spills in the
@@ -1004,10 +1050,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kTileCopies) ok = masked ? tile(std::true_type{}) : tile(std::false_type{});
         else ok = tile(!ALIBI && masked);
         if (!ok) break;
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_ready[t]);
-        if (tracer) MEA_TRACE_AT(t * 512 + j * 16 + 4);
+        if constexpr (kSepP) {
+          tmem_st_wait();
+          tc_fence_before();
+          warp_arrive(&p_ready[4 * t]);
+        }
+        if (tracer) MEA_TRACE_AT(t * 4096 + (nc & 255) * 16 + 4);
+        if (lane == 0) MEA_TRACE_AT(13632 + (warp & 15) * 256 + (nc & 255));
         ++nc;
       }
       if constexpr (!SPARSE) nc = nbase + ntt;
@@ -1055,6 +1104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (tracer && t == 0 && ku == 0) MEA_CTA_AT(3);
+      if (tracer) MEA_TRACE_AT(12288 + (ku & 63) * 4 + 2 * t + 1);
       return ok;
     });
   }
