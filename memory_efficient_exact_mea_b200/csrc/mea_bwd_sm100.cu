@@ -103,18 +103,20 @@ struct BwdCfg {
   static constexpr int kKVTile = kChunksD * kKVChunk;
   static constexpr int kQTile = kChunksD * kQChunk;
   static constexpr int kDSTile = (BM / 64) * kKVChunk;  // dS^T: 128 keys x BM queries
-  // Q / dO stages: three at K = 128; two at K = 64, where a third does not fit
-  // beside the dQ staging buffer.
-  static constexpr int kStages = (D == 128) ? 3 : 2;
+  // Q / dO stages: three (two steps of look-ahead for the loads).
+  static constexpr int kStages = 3;
   static constexpr int kStage = 2 * kQTile;           // Q then dO
-  static constexpr int kDQSBox = BM * 128;            // dQ staging: D/32 boxes of BM x 128 B
+  static constexpr int kDQSBox = BM * 128;            // dQ staging: boxes of BM x 128 B
+  // K = 128 stages all D/32 boxes of a step at once; K = 64 (BM = 128) one box at a
+  // time, which leaves room for the third Q / dO stage.
+  static constexpr int kDQSBoxes = (D == 128) ? D / 32 : 1;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kK = 0;
   static constexpr int kV = kKVTile;
   static constexpr int kQD = 2 * kKVTile;              // stage i: Q at kQD + i*kStage, dO after it
   static constexpr int kDS = kQD + kStages * kStage;   // two buffers (step parity)
   static constexpr int kDQS = kDS + 2 * kDSTile;       // dQ of one step, fp32, for the reductions
-  static constexpr int kLse = kDQS + (D / 32) * kDQSBox;  // [stage][BM] -lse * log2(e) (-inf: no weight)
+  static constexpr int kLse = kDQS + kDQSBoxes * kDQSBox;  // [stage][BM] -lse * log2(e) (-inf: no weight)
   static constexpr int kDelta = kLse + kStages * BM * 4;  // [stage][BM] -D
   static constexpr int kBar = kDelta + kStages * BM * 4;
   static constexpr int kNumBars = 14;
@@ -255,11 +257,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 256);
-    mbar_init(p_ready, 256);
+    mbar_init(s_free, 8);  // one arrival per P/dS warp
+    mbar_init(p_ready, 8);
     mbar_init(p_done, 1);
     mbar_init(dq_full, 1);
-    mbar_init(dq_empty, 128);
+    mbar_init(dq_empty, 4);  // one arrival per dQ drain warp
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -340,8 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(&q_full[s % NS], (s / NS) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
-    // ===================== MMA issue (one thread) ============================
-    if (lane == 0) {
+    // ===================== MMA issue (one warp) ==============================
+    // The whole warp runs the loop (all values warp-uniform); elect.sync picks the
+    // lane that issues each MMA and commit.
+    {
       constexpr uint32_t idesc_s = idesc_f16_ab(BF16, kBN, BM, false, false);
       constexpr uint32_t idesc_g = idesc_f16_ab(BF16, kBN, D, false, true);
       constexpr uint32_t idesc_q = idesc_f16_ab(BF16, kBN, 64, true, true);
@@ -360,20 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::kKVChunk + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
-          umma_ss(tS, sdesc_sw128(sK + okv, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), idesc_s,
+          umma_ss_warp(tS, sdesc_sw128(sK + okv, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), idesc_s,
                   kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::kKVChunk + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * C::kQChunk + (kk & 3) * 32;
-          umma_ss(tDP, sdesc_sw128(sV + okv, 16, 1024), sdesc_sw128(sDO + oq, 16, 1024), idesc_s,
+          umma_ss_warp(tDP, sdesc_sw128(sV + okv, 16, 1024), sdesc_sw128(sDO + oq, 16, 1024), idesc_s,
                   kk > 0);
         }
-        umma_commit(s_full);
+        umma_commit_warp(s_full);
       };
-      bool ok = steps > 0 && mbar_wait(kv_full, 0, abort_flag, a.status) &&
-                mbar_wait(&q_full[0], 0, abort_flag, a.status);
+      bool ok = steps > 0 && mbar_wait_warp(kv_full, 0, abort_flag, a.status) &&
+                mbar_wait_warp(&q_full[0], 0, abort_flag, a.status);
       if (ok) {
         BWD_TRACE_CTA(1);
         tc_fence_after();
@@ -384,16 +388,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The next block's scores go first: they only need its Q / dO and the
         // S^T / dP^T columns, which the P/dS threads have read out.
         if (s + 1 < steps) {
-          if (!(ok = mbar_wait(&q_full[(s + 1) % NS], ((s + 1) / NS) & 1, abort_flag, a.status)))
+          if (!(ok = mbar_wait_warp(&q_full[(s + 1) % NS], ((s + 1) / NS) & 1, abort_flag, a.status)))
             break;
           BWD_TRACE(s, 0);
-          if (!(ok = mbar_wait(s_free, s & 1, abort_flag, a.status))) break;
+          if (!(ok = mbar_wait_warp(s_free, s & 1, abort_flag, a.status))) break;
           BWD_TRACE(s, 1);
           tc_fence_after();
           issue_s(s + 1);
           BWD_TRACE(s, 2);
         }
-        if (!(ok = mbar_wait(p_ready, s & 1, abort_flag, a.status))) break;
+        if (!(ok = mbar_wait_warp(p_ready, s & 1, abort_flag, a.status))) break;
         BWD_TRACE(s, 3);
         tc_fence_after();
         const uint32_t sQ = smem_u32(smem + C::kQD + slot * C::kStage);
@@ -403,21 +407,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dO and Q as N-contiguous B operands, 16 query rows (2048 bytes) per step.
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tDV, tP + kk * 8, sdesc_sw128(sDO + kk * 2048, C::kQChunk, 1024), idesc_g,
+          umma_ts_warp(tDV, tP + kk * 8, sdesc_sw128(sDO + kk * 2048, C::kQChunk, 1024), idesc_g,
                   (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ss(tDK, sdesc_sw128(sDS + (kk >> 2) * C::kKVChunk + (kk & 3) * 32, 16, 1024),
+          umma_ss_warp(tDK, sdesc_sw128(sDS + (kk >> 2) * C::kKVChunk + (kk & 3) * 32, 16, 1024),
                   sdesc_sw128(sQ + kk * 2048, C::kQChunk, 1024), idesc_g,
                   (s > 0 || kk > 0) ? 1u : 0u);
         // No later MMA reads this step's Q / dO stage: the loader may refill it
         // once these have completed.
-        umma_commit(&q_empty[slot]);
+        umma_commit_warp(&q_empty[slot]);
         // dQ: both operands M/N-contiguous views of row-major 128-key tiles, 16 keys
         // (2048 bytes) per step.  K = 128: dQ^T = K^T dS^T; K = 64: dQ = dS K.
         BWD_TRACE(s, 4);
         if (s > 0) {
-          if (!(ok = mbar_wait(dq_empty, (s - 1) & 1, abort_flag, a.status))) break;
+          if (!(ok = mbar_wait_warp(dq_empty, (s - 1) & 1, abort_flag, a.status))) break;
           tc_fence_after();
         }
         BWD_TRACE(s, 5);
@@ -425,14 +429,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t qb = (D == 128) ? sDS : sK;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ss(tDQ, sdesc_sw128(qa + kk * 2048, C::kKVChunk, 1024),
+          umma_ss_warp(tDQ, sdesc_sw128(qa + kk * 2048, C::kKVChunk, 1024),
                   sdesc_sw128(qb + kk * 2048, C::kKVChunk, 1024), idesc_q, kk > 0);
-        umma_commit(dq_full);
-        umma_commit(p_done);
+        umma_commit_warp(dq_full);
+        umma_commit_warp(p_done);
         BWD_TRACE(s, 6);
       }
       // Every MMA issued above has completed once this barrier flips.
-      umma_commit(mma_done);
+      umma_commit_warp(mma_done);
       mbar_wait_drain(mma_done, 0, a.status);
     }
   } else if (warp < 8) {
@@ -457,10 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = s % NS;
       float slope_log2 = 0.f;
       if constexpr (ALIBI) slope_log2 = exp2f(-8.0f * static_cast<float>(h + 1) / a.Hq) * kLog2e;
+      const bool tracer = warp == 0 && lane == 0;
+      if (tracer) BWD_TRACE(s, 13);
       // -lse / -D of this block were staged with the Q copy of the stage.
       if (!(ok = mbar_wait_warp(&q_full[slot], (s / NS) & 1, abort_flag, a.status))) break;
+      if (tracer) BWD_TRACE(s, 14);
       if (!(ok = mbar_wait_warp(s_full, s & 1, abort_flag, a.status))) break;
-      const bool tracer = warp == 0 && lane == 0;
       if (tracer) BWD_TRACE(s, 8);
       tc_fence_after();
       // Per-element masks only where the tile reaches past the keys or past the
@@ -487,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait(dr);
           if (c == kCols / 32 - 1) {
             tc_fence_before();
-            mbar_arrive(s_free);  // the next block's S^T / dP^T may be written now
+            mbar_arrive_warp(s_free);  // the next block's S^T / dP^T may be written now
             if (tracer) BWD_TRACE(s, 9);
           }
 #pragma unroll
@@ -497,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 dd = *reinterpret_cast<const float2*>(nd + k);
             f2 x = fma2(f2{__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])}, scale2,
                         f2{l.x, l.y});
-            const int pos = m0 + c0 + k + off;  // query position of column k, key coordinates
+            [[maybe_unused]] const int pos = m0 + c0 + k + off;  // query position of column k, key coordinates
             if constexpr (ALIBI) {
               x.x -= slope_log2 * fabsf(static_cast<float>(pos - j_loc));
               x.y -= slope_log2 * fabsf(static_cast<float>(pos + 1 - j_loc));
@@ -546,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive_warp(p_ready);
       if (tracer) BWD_TRACE(s, 12);
     }
     // ---- epilogue: dK (scaled) and dV of the valid keys, half of K each -------
@@ -606,18 +612,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait_warp(dq_full, s & 1, abort_flag, a.status))) break;
       if (leader) BWD_TRACE(s, 16);
       tc_fence_after();
-      // Stage dQ in the staging buffer, once the previous step's reductions have
-      // read it (the leader waits for them, then joins this barrier).
+      // Stage dQ in the staging buffer, once the previous reductions have read it
+      // (the leader waits for them, then joins barrier 2).  K = 128: all boxes,
+      // then their reductions; K = 64: one 32-column box at a time.
       uint8_t* stage = smem + C::kDQS;
-      if (s > 0) named_sync(2, 128);
+      constexpr bool kOneBox = C::kDQSBoxes == 1;
+      auto reduce = [&](int b0, int nb) {
+        fence_async_smem();
+        named_sync(1, 128);
+        if (leader) {
+          BWD_TRACE(s, 17);
+          for (int b = b0; b < b0 + nb; ++b)
+            tma_reduce_add_4d(&tmDQ, stage + (kOneBox ? 0 : b * C::kDQSBox), 32 * b, h, q0 + m0,
+                              bidx);
+          bulk_commit();
+          bulk_wait_read();  // the staging buffer may be written again
+        }
+      };
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
+        if (kOneBox ? (s > 0 || half > 0) : (s > 0 && half == 0)) named_sync(2, 128);
         uint32_t v[32];
         tmem_ld32(t_addr + 32 * half, v);
         tmem_ld_wait(v);
         if (half == 1) {
           tc_fence_before();
-          mbar_arrive(dq_empty);
+          mbar_arrive_warp(dq_empty);
         }
         if constexpr (D == 128) {
           // lane = dimension `row`, columns = queries 32 half .. +31: element
@@ -634,24 +654,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           // lane = query m0 + row, columns = dims 32 half .. +31 = box `half`:
           // 16-byte piece u at u ^ (row & 7).
           const float sc = (m0 + row < q_len) ? a.scale : 0.f;
-          uint8_t* line = stage + half * C::kDQSBox + row * 128;
+          uint8_t* line = stage + row * 128;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<float4*>(line + ((u ^ (row & 7)) << 4)) =
                 make_float4(__uint_as_float(v[4 * u]) * sc, __uint_as_float(v[4 * u + 1]) * sc,
                             __uint_as_float(v[4 * u + 2]) * sc, __uint_as_float(v[4 * u + 3]) * sc);
+          reduce(half, 1);
         }
       }
-      fence_async_smem();
-      named_sync(1, 128);
-      if (leader) {
-        BWD_TRACE(s, 17);
-#pragma unroll
-        for (int b = 0; b < D / 32; ++b)
-          tma_reduce_add_4d(&tmDQ, stage + b * C::kDQSBox, 32 * b, h, q0 + m0, bidx);
-        bulk_commit();
-        bulk_wait_read();  // the staging buffer may be written again
-      }
+      if constexpr (!kOneBox) reduce(0, D / 32);
     }
     if (leader) bulk_wait_all();
   }

@@ -90,10 +90,11 @@ __device__ __forceinline__ int opaque(int x) {
 // issuing thread) or 8192 + t*2048 + l*8 + e (one per tile); unit k (modulo 64),
 // softmax tile t -> 12288 + k*4 + 2t (start), + 1 (epilogue done); TMA ring copy
 // i (modulo 512) issued -> 12544 + 2i; Q load of unit k (modulo 64) -> 13568 + k;
-// softmax warp w, step n: P published -> 13632 + w*256 + n.
+// softmax warp w, step n: P published -> 13632 + w*256 + n; epilogue of unit k,
+// tile t: O complete, O read, rows stored -> 17728 + k*8 + 4t + (0, 1, 2).
 #ifdef MEA_TRACE
 constexpr int kTraceCtas = 4;
-constexpr int kTraceSlots = 17728;
+constexpr int kTraceSlots = 18240;
 __device__ long long g_trace[kTraceCtas * kTraceSlots];
 #define MEA_TRACE_AT(slot)                                                         \
   do {                                                                             \
@@ -1070,6 +1071,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 2; ++e) rr[e] = opaque(m_base + t * kBM + lane0 + t1 + 8 * e);
       }
       if (ok && nc > nbase) ok = mbar_wait_warp(&o_done[t], (nc - 1) & 1, abort_flag, a.status);
+      if (tracer) MEA_TRACE_AT(17728 + (ku & 63) * 8 + 4 * t);
       if (ok) {
         tc_fence_after();
         float l_tot[2];
@@ -1085,6 +1087,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kOReg; ++i) o[i] = 0u;
         }
+        if (tracer) MEA_TRACE_AT(17728 + (ku & 63) * 8 + 4 * t + 1);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           if (rr[e] >= q_len) continue;
@@ -1104,6 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (tracer && t == 0 && ku == 0) MEA_CTA_AT(3);
+      if (tracer) MEA_TRACE_AT(17728 + (ku & 63) * 8 + 4 * t + 2);
       if (tracer) MEA_TRACE_AT(12288 + (ku & 63) * 4 + 2 * t + 1);
       return ok;
     });
