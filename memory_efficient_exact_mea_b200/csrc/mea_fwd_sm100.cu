@@ -167,6 +167,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kPersist = kPersistent<D, BF16, MASK, ALIBI, MODE>;
   constexpr bool kCausal = (MASK == 1 || MASK == 3);
   constexpr bool kPacked = (MASK >= 2);
+  // Causal instances without a cache walk a unit's key tiles from the diagonal
+  // back to the first: keys nearer the query come first, and with ALiBi, whose
+  // bias falls with distance, the first tile then holds (nearly always) the row's
+  // largest logits, so the running max rarely moves afterwards and the output is
+  // rarely rescaled.  Each query tile computes a suffix of the unit's steps.
+  constexpr bool kDesc = kCausal && MODE == kModeDense;
   constexpr bool kSplitP = BF16;  // P.V as (P_hi + P_lo).V for bf16
   // With K = 64 and fp16, P gets TMEM columns of its own (S 2x128, P 2x64, O 2x64
   // = 512), so S_t is free as soon as the softmax has read it and the next
@@ -451,13 +457,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = last ? q_len - kBN : m * kBN;
       return {r, past + r, last ? n_new_tiles * kBN - q_len : 0, true};
     }
-    return {k0 + j * kBN, j * kBN, 0, false};
+    const int jk = kDesc ? nt - 1 - j : j;  // the key tile of step j
+    return {k0 + jk * kBN, jk * kBN, 0, false};
   };
 
   // Does query tile t compute key tile j?  Every role walks the key tiles in
   // the same order and skips those neither query tile needs; the barriers of a
   // query tile count only the key tiles that tile computes.
   auto uses = [&](int t, int j) -> bool {
+    if constexpr (kDesc) return j >= nt - nt_tile[t];
     if (j >= nt_tile[t]) return false;
     if constexpr (SPARSE) return __ldg(t ? mrow1 + j : mrow0 + j) != 0;
     return true;
@@ -647,8 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (SPARSE) {
               if (!used && !uses(1 - t, j)) continue;
             } else {
-              li = li0 + j;  // dense: every key tile is in the ring and a tile uses a prefix
-              c = c0 + j;
+              // dense: every key tile is in the ring and a tile uses a prefix of the
+              // steps (a suffix when walking down from the diagonal)
+              li = li0 + j;
+              c = c0 + (kDesc ? max(0, j - (nt - nt_tile[t])) : j);
             }
             const int ks = (2 * li) % S;
             if (!(ok = mbar_wait_warp(&kv_full[ks], ((2 * li) / S) & 1, abort_flag, a.status))) break;
@@ -704,10 +714,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (SPARSE) {
               if (!u0 && !u1) continue;
             } else {  // dense: every key tile is in the ring and each tile uses a prefix
-              li = li0 + j;
+              li = li0 + j;  // (a suffix when walking down from the diagonal)
               it = 2 * li;
-              c0 = c00 + j;
-              c1 = c10 + j;
+              c0 = c00 + (kDesc ? max(0, j - (nt - nt_tile[0])) : j);
+              c1 = c10 + (kDesc ? max(0, j - (nt - nt_tile[1])) : j);
             }
             const int kslot = it % S;
             if (!(ok = mbar_wait_warp(&kv_full[kslot], (it / S) & 1, abort_flag, a.status))) break;
@@ -835,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tracer && t == 0 && j == 0 && ku == 0) MEA_CTA_AT(1);
         // Keys this row may see in the tile: columns [kfirst, limit).  Tiles that
         // need no masking for any row of the warp take the unmasked path.
-        int n0 = j * kBN, kfirst = 0;
+        int n0 = (kDesc ? ntt - 1 - j : j) * kBN, kfirst = 0;
         if constexpr (kCache) {
           const KeyTile kt = key_tile(j);
           n0 = kt.pos;

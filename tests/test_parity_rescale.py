@@ -16,6 +16,9 @@ leave the first tile's reference.  The inputs here do:
   steps    scores constant per 128-key tile, moving by exactly 8, 7.9375,
            8.0625, ... log2 units from tile to tile (scale = ln 2, so a score is
            its log2 logit), around the threshold where the reference moves.
+Dense causal instances walk a unit's key tiles from the diagonal down, so for
+them "falling" is the shape whose maximum climbs; the step shapes run with both
+signs.
 Every instance family without ALiBi is covered (ALiBi's growing bias already
 moves the maximum): the persistent K=64 fp16 non-causal instance with more
 units than SMs, K=64 fp16 causal (P in its own tensor-memory columns), K=128
@@ -112,14 +115,18 @@ STEP_CASES = [(64, "f16", "none"), (64, "f16", "causal"), (128, "bf16", "none"),
               (128, "bf16", "causal"), (64, "bf16", "none"), (128, "f16", "causal")]
 
 
+@pytest.mark.parametrize("sign", [1.0, -1.0])
 @pytest.mark.parametrize("noise", [0.0, 0.05])
 @pytest.mark.parametrize("K,dtype,bias", STEP_CASES)
-def test_threshold_steps(mea, orc, K, dtype, bias, noise):
+def test_threshold_steps(mea, orc, K, dtype, bias, noise, sign):
     """Tile-to-tile jumps of exactly 8 (kept stale: P reaches 2^8), 7.9375 (kept),
     8.0625 (moved), a fall of 30 and a rise of 16, in rotated orders per batch;
-    with noise the rows straddle the threshold differently."""
-    p = synth.tile_step_scores(f"steps_{K}_{dtype}_{bias}_n{noise}", 3, 1100, 2, K, dtype,
-                               STEPS, 128, seed=520 + K, bias=bias, noise=noise)
+    with noise the rows straddle the threshold differently.  The negated steps
+    give the same jumps to a kernel that walks the key tiles downwards (dense
+    causal instances)."""
+    steps = [sign * s for s in STEPS]
+    p = synth.tile_step_scores(f"steps_{K}_{dtype}_{bias}_n{noise}_s{sign:+.0f}", 3, 1100, 2, K,
+                               dtype, steps, 128, seed=520 + K, bias=bias, noise=noise)
     _check_dense(mea, orc, p, LN2_F32)
 
 
