@@ -23,10 +23,9 @@
 //     P^T (16-bit) to its own TMEM columns, dS^T to shared memory (two buffers)
 //   dV  += P^T dO_i   (A = P^T from TMEM)              dK += dS^T Q_i
 //   dQ_i = dS_i K  (K = 64)  or  dQ_i^T = K^T dS_i^T (K = 128): both M = 128, N = 64
-//   dQ_i is drained by four warps: scaled, staged in shared memory -- in the
-//   Q_i/dO_i stage, which no MMA reads any more -- and added to the fp32
-//   accumulator by TMA tensor reductions (one per 32 columns); the stage is
-//   handed back to the loader once the reductions have read it.
+//   dQ_i is drained by four warps: scaled, staged in a shared-memory buffer of its
+//   own and added to the fp32 accumulator by TMA tensor reductions (one per 32
+//   columns).
 // The S^T / dP^T columns are released as soon as the P/dS threads have read
 // them, so the MMA thread issues the next block's S^T, dP^T before this block's
 // dV, dK, dQ and the P/dS arithmetic of one block overlaps the MMAs of its
@@ -35,8 +34,8 @@
 // is stored once block i-1's MMAs are done.
 //
 // CTA (448 threads): warps 0-7 P/dS and the dK/dV epilogue (warps w and w+4
-// share TMEM lane quarter w, each taking half of the query columns), warps 8-11
-// the dQ drain, warp 12 allocates TMEM and one of its threads issues every MMA,
+// share TMEM lane quarter w, each taking half of the query columns, read 16 at a
+// time), warps 8-11 the dQ drain, warp 12 allocates TMEM and issues every MMA,
 // warp 13 loads (one thread issues the TMA copies; the warp stages lse and D).
 #include <math.h>
 
@@ -51,14 +50,17 @@ namespace mea {
 namespace {
 
 constexpr int kBN = kBwdBlock;  // keys per CTA (= TMEM lanes)
-constexpr int kThreads = 448;
-constexpr int kDrainWarp = 8;  // warps 8..11
-constexpr int kMmaWarp = 12;
-constexpr int kLoadWarp = 13;
+constexpr int kPdsWarps = 8;  // P/dS warps: two per TMEM lane quarter (a column half each)
+constexpr int kThreads = (kPdsWarps + 6) * 32;
+constexpr int kDrainWarp = kPdsWarps;  // four drain warps
+constexpr int kMmaWarp = kPdsWarps + 4;
+constexpr int kLoadWarp = kPdsWarps + 5;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+
 
 // Pipeline timeline for performance work: built only with -DMEA_TRACE, it
 // records clock64() at pipeline events of the first kBwdTraceCtas CTAs.
@@ -257,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 8);  // one arrival per P/dS warp
-    mbar_init(p_ready, 8);
+    mbar_init(s_free, kPdsWarps);  // one arrival per P/dS warp
+    mbar_init(p_ready, kPdsWarps);
     mbar_init(p_done, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 4);  // one arrival per dQ drain warp
@@ -439,12 +441,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit_warp(mma_done);
       mbar_wait_drain(mma_done, 0, a.status);
     }
-  } else if (warp < 8) {
+  } else if (warp < kPdsWarps) {
     // ===================== P^T and dS^T, then the dK / dV epilogue ============
-    constexpr int kCols = BM / 2;  // query columns per thread
-    const int quarter = warp & 3, half = warp >> 2;
+    constexpr int kParts = kPdsWarps / 4;  // warps sharing a TMEM lane quarter
+    constexpr int kCols = BM / kParts;     // query columns per thread (32 at K = 64, 16 at 128)
+    const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;  // key inside the block = TMEM lane
-    const int c0 = half * kCols;          // this thread's first query column
+    const int c0 = part * kCols;          // this thread's first query column
     const int j_loc = n0 + row;
     const bool key_ok = j_loc < k_len;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -482,23 +485,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // only, through c0, as the warp-collective TMEM loads inside require).
       // K = 64: one copy with a run-time test (two copies spill there).
       auto p_ds = [&](auto msk) {
-        // 32 columns at a time: read S^T, dP^T out of TMEM (releasing them after the
-        // last chunk), then P = 2^(s*scale*log2e - lse*log2e) and dS = P (dP - D).
+        // kChunk columns at a time: read S^T, dP^T out of TMEM (releasing them after
+        // the last chunk), then P = 2^(s*scale*log2e - lse*log2e) and dS = P (dP - D).
+        constexpr int kChunk = 16;
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          uint32_t sr[32], dr[32], dk[16];
-          tmem_ld32(tS + 32 * c, sr);
-          tmem_ld32(tDP + 32 * c, dr);
-          tmem_ld_wait(sr);
-          tmem_ld_wait(dr);
-          if (c == kCols / 32 - 1) {
+        for (int c = 0; c < kCols / kChunk; ++c) {
+          uint32_t sr[kChunk], dr[kChunk], dk[kChunk / 2];
+          tmem_ld2x16_wait(tS + kChunk * c, tDP + kChunk * c, sr, dr);
+          if (c == kCols / kChunk - 1) {
             tc_fence_before();
             mbar_arrive_warp(s_free);  // the next block's S^T / dP^T may be written now
             if (tracer) BWD_TRACE(s, 9);
           }
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int k = 32 * c + e;
+          for (int e = 0; e < kChunk; e += 2) {
+            const int k = kChunk * c + e;
             const float2 l = *reinterpret_cast<const float2*>(nl + k);
             const float2 dd = *reinterpret_cast<const float2*>(nd + k);
             f2 x = fma2(f2{__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])}, scale2,
@@ -524,12 +525,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[k / 2] = pack2<BF16>(p.x, p.y);
             dk[e / 2] = pack2<BF16>(ds.x, ds.y);
           }
-          // dS^T row `row`, columns c0+32c .. +31, in the 128-byte-swizzled layout the
-          // MMA descriptors read: 16-byte piece u of a 64-column chunk sits at u ^ (row & 7).
-          const int col = c0 + 32 * c;
+          // dS^T row `row`, columns c0 + kChunk c .. + kChunk - 1, in the 128-byte-swizzled
+          // layout the MMA descriptors read: 16-byte piece u of a 64-column chunk sits at
+          // u ^ (row & 7).
+          const int col = c0 + kChunk * c;
           const int plane = col >> 6;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < kChunk / 8; ++u) {
             const int piece = ((col & 63) >> 3) + u;
             *reinterpret_cast<uint4*>(ds_buf + plane * C::kKVChunk + ((piece ^ (row & 7)) << 4)) =
                 make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
@@ -547,57 +549,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (s > 0 && !(ok = mbar_wait_warp(p_done, (s - 1) & 1, abort_flag, a.status))) break;
       if (tracer) BWD_TRACE(s, 11);
       tc_fence_after();
+      if constexpr (kCols == 16) {
+        tmem_st8(tP, pk);  // 16 queries, two per column
+      } else {
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
+        for (int c = 0; c < kCols / 32; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
+      }
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();
       mbar_arrive_warp(p_ready);
       if (tracer) BWD_TRACE(s, 12);
     }
-    // ---- epilogue: dK (scaled) and dV of the valid keys, half of K each -------
+    // ---- epilogue: dK (scaled) and dV of the valid keys, D / kParts columns each --
     // The TMEM loads are warp-collective: every lane issues them, and only the
     // global stores depend on the lane's key.
     if (ok) ok = mbar_wait_warp(mma_done, 0, abort_flag, a.status);
     if (warp == 0 && lane == 0) BWD_TRACE_CTA(2);
     if (ok) {
       tc_fence_after();
-      const int dc0 = half * (D / 2);
+      const int dc0 = part * (D / kParts);
       const long long grow = (static_cast<long long>(bidx) * a.N + k0 + j_loc) * a.Hkv + kvh;
       uint8_t* dk_row = static_cast<uint8_t*>(a.dk) + (grow * D + dc0) * 2;
       uint8_t* dv_row = static_cast<uint8_t*>(a.dv) + (grow * D + dc0) * 2;
 #pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t kr[32], vr[32];
+      for (int c = 0; c < D / kParts / 16; ++c) {
+        uint32_t kr[16], vr[16];
         if (steps > 0) {
-          tmem_ld32(tmem_base + lane_addr + C::kColDK + dc0 + 32 * c, kr);
-          tmem_ld32(tmem_base + lane_addr + C::kColDV + dc0 + 32 * c, vr);
-          tmem_ld_wait(kr);
-          tmem_ld_wait(vr);
+          tmem_ld2x16_wait(tmem_base + lane_addr + C::kColDK + dc0 + 16 * c,
+                           tmem_base + lane_addr + C::kColDV + dc0 + 16 * c, kr, vr);
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) kr[i] = vr[i] = 0u;
+          for (int i = 0; i < 16; ++i) kr[i] = vr[i] = 0u;
         }
-        uint32_t pkk[16], pkv[16];
+        uint32_t pkk[8], pkv[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
           pkk[i] = pack2<BF16>(__uint_as_float(kr[2 * i]) * a.scale,
                                __uint_as_float(kr[2 * i + 1]) * a.scale);
           pkv[i] = pack2<BF16>(__uint_as_float(vr[2 * i]), __uint_as_float(vr[2 * i + 1]));
         }
         if (key_ok) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            reinterpret_cast<uint4*>(dk_row + c * 64)[u] =
+          for (int u = 0; u < 2; ++u) {
+            reinterpret_cast<uint4*>(dk_row + c * 32)[u] =
                 make_uint4(pkk[4 * u], pkk[4 * u + 1], pkk[4 * u + 2], pkk[4 * u + 3]);
-            reinterpret_cast<uint4*>(dv_row + c * 64)[u] =
+            reinterpret_cast<uint4*>(dv_row + c * 32)[u] =
                 make_uint4(pkv[4 * u], pkv[4 * u + 1], pkv[4 * u + 2], pkv[4 * u + 3]);
           }
         }
       }
     }
   } else {
-    // ===================== dQ drain (warps 8-11) ==============================
+    // ===================== dQ drain (warps 16-19) =============================
     // dQ of a step goes TMEM -> registers (scaled) -> a 128-byte-swizzled staging
     // tile in shared memory, whose 32-column boxes are added to the fp32
     // accumulator by TMA reductions issued by one thread.
@@ -629,28 +633,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_wait_read();  // the staging buffer may be written again
         }
       };
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
-        if (kOneBox ? (s > 0 || half > 0) : (s > 0 && half == 0)) named_sync(2, 128);
-        uint32_t v[32];
-        tmem_ld32(t_addr + 32 * half, v);
-        tmem_ld_wait(v);
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive_warp(dq_empty);
-        }
-        if constexpr (D == 128) {
-          // lane = dimension `row`, columns = queries 32 half .. +31: element
-          // (query q, dim row) of box row/32 at row q, byte 4 (row % 32), swizzled.
-          uint8_t* box = stage + (row >> 5) * C::kDQSBox;
-          const int piece = (row & 31) >> 2, word = (row & 3) * 4;
+      if constexpr (D == 64) {
+        // Both 32-column halves come out of TMEM first, so dQ's columns are handed
+        // back before the one-box-at-a-time staging and reductions.
+        uint32_t v0[32], v1[32];
+        tmem_ld32(t_addr, v0);
+        tmem_ld32(t_addr + 32, v1);
+        tmem_ld_wait(v0);
+        tmem_ld_wait(v1);
+        tc_fence_before();
+        mbar_arrive_warp(dq_empty);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int q = 32 * half + k;
-            const float x = (m0 + q < q_len) ? __uint_as_float(v[k]) * a.scale : 0.f;
-            *reinterpret_cast<float*>(box + q * 128 + ((piece ^ (k & 7)) << 4) + word) = x;
-          }
-        } else {
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t(&v)[32] = half ? v1 : v0;
+          if (s > 0 || half > 0) named_sync(2, 128);
           // lane = query m0 + row, columns = dims 32 half .. +31 = box `half`:
           // 16-byte piece u at u ^ (row & 7).
           const float sc = (m0 + row < q_len) ? a.scale : 0.f;
@@ -662,8 +658,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __uint_as_float(v[4 * u + 2]) * sc, __uint_as_float(v[4 * u + 3]) * sc);
           reduce(half, 1);
         }
+      } else {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
+          if (s > 0 && half == 0) named_sync(2, 128);
+          uint32_t v[32];
+          tmem_ld32(t_addr + 32 * half, v);
+          tmem_ld_wait(v);
+          if (half == 1) {
+            tc_fence_before();
+            mbar_arrive_warp(dq_empty);
+          }
+          // lane = dimension `row`, columns = queries 32 half .. +31: element
+          // (query q, dim row) of box row/32 at row q, byte 4 (row % 32), swizzled.
+          uint8_t* box = stage + (row >> 5) * C::kDQSBox;
+          const int piece = (row & 31) >> 2, word = (row & 3) * 4;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int q = 32 * half + k;
+            const float x = (m0 + q < q_len) ? __uint_as_float(v[k]) * a.scale : 0.f;
+            *reinterpret_cast<float*>(box + q * 128 + ((piece ^ (k & 7)) << 4) + word) = x;
+          }
+        }
+        reduce(0, D / 32);
       }
-      if constexpr (!kOneBox) reduce(0, D / 32);
     }
     if (leader) bulk_wait_all();
   }
