@@ -37,6 +37,8 @@
 // share TMEM lane quarter w, each taking half of the query columns, read 16 at a
 // time), warps 8-11 the dQ drain, warp 12 allocates TMEM and issues every MMA,
 // warp 13 loads (one thread issues the TMA copies; the warp stages lse and D).
+// The MMA warp runs its issuing loop warp-wide; elect.sync picks the lane that
+// issues each MMA and commit.
 #include <math.h>
 
 #include <algorithm>
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kPdsWarps) {
     // ===================== P^T and dS^T, then the dK / dV epilogue ============
     constexpr int kParts = kPdsWarps / 4;  // warps sharing a TMEM lane quarter
-    constexpr int kCols = BM / kParts;     // query columns per thread (32 at K = 64, 16 at 128)
+    constexpr int kCols = BM / kParts;     // query columns per thread (64 at K = 64, 32 at 128)
     const int quarter = warp & 3, part = warp >> 2;
     const int row = quarter * 32 + lane;  // key inside the block = TMEM lane
     const int c0 = part * kCols;          // this thread's first query column
@@ -549,12 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (s > 0 && !(ok = mbar_wait_warp(p_done, (s - 1) & 1, abort_flag, a.status))) break;
       if (tracer) BWD_TRACE(s, 11);
       tc_fence_after();
-      if constexpr (kCols == 16) {
-        tmem_st8(tP, pk);  // 16 queries, two per column
-      } else {
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
-      }
+      for (int c = 0; c < kCols / 32; ++c) tmem_st16(tP + 16 * c, pk + 16 * c);
       tmem_st_wait();
       fence_async_smem();
       tc_fence_before();

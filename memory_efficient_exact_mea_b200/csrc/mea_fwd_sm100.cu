@@ -14,10 +14,12 @@
 //               each warp on 16 lanes of its lane quarter, four threads per row
 //               (a quarter of the columns each) in one warp
 //   warps 8-15  the same for query tile 1 (rows +128)
-//   warp  16    TMEM allocator; one thread issues every MMA of query tile 0 (and,
-//               with P written over S, of query tile 1 too, interleaved)
-//   warp  17    separate-P layout: one thread issues every MMA of query tile 1
-//               (the two tiles do not wait for each other)
+//   warp  16    TMEM allocator; issues every MMA of query tile 0 (and, with P
+//               written over S, of query tile 1 too, interleaved)
+//   warp  17    separate-P layout: issues every MMA of query tile 1 (the two
+//               tiles do not wait for each other); both issuers run their loops
+//               warp-wide, elect.sync picking the lane that executes each
+//               tcgen05.mma and tcgen05.commit
 //   warp  18    the single TMA-issuing thread
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, the scores of the
 // current key tile; P = exp(S - m) as 16-bit pairs is written back over S, each
