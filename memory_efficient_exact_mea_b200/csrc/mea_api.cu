@@ -465,7 +465,7 @@ extern "C" int mea_bwd_stages(const void* q, const void* k, const void* v, const
         !encode_bmhk(&L.tmDO, dout, bf16, B, M, Hq, K, sq, bm) ||
         !encode_bmhk(&L.tmK, k, bf16, B, N, Hkv, K, sk, mea::kBwdBlock) ||
         !encode_bmhk(&L.tmV, v, bf16, B, N, Hkv, K, sk, mea::kBwdBlock) ||
-        !encode_f32_bmhk(&L.tmDQ, workspace, B, M, Hq, K, bm))
+        !encode_f32_bmhk(&L.tmDQ, workspace, B, M, Hq, K, mea::bwd_dq_box_rows(K)))
       return MEA_ERR_CUDA;
   }
   mea::BwdArgs& a = L.args;

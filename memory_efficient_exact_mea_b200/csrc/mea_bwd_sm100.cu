@@ -62,6 +62,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 
+// Wait until every bulk async-group of this thread but the most recent one has
+// finished reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 
 
 // Pipeline timeline for performance work: built only with -DMEA_TRACE, it
@@ -110,10 +116,14 @@ struct BwdCfg {
   // Q / dO stages: three (two steps of look-ahead for the loads).
   static constexpr int kStages = 3;
   static constexpr int kStage = 2 * kQTile;           // Q then dO
-  static constexpr int kDQSBox = BM * 128;            // dQ staging: boxes of BM x 128 B
-  // K = 128 stages all D/32 boxes of a step at once; K = 64 (BM = 128) one box at a
-  // time, which leaves room for the third Q / dO stage.
-  static constexpr int kDQSBoxes = (D == 128) ? D / 32 : 1;
+  // dQ staging, in boxes of kDQRows rows x 32 fp32 (128 B a row).  K = 128: the
+  // D/32 boxes of one half step (32 queries) at a time, in two buffers, so one
+  // half is staged while the other's reductions read it; K = 64 (BM = 128): one
+  // 32-dimension box of the step at a time, which leaves room for the third Q / dO
+  // stage.
+  static constexpr int kDQRows = (D == 128) ? 32 : BM;
+  static constexpr int kDQSBox = kDQRows * 128;
+  static constexpr int kDQSBoxes = (D == 128) ? 2 * (D / 32) : 1;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kK = 0;
   static constexpr int kV = kKVTile;
@@ -615,18 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) BWD_TRACE(s, 16);
       tc_fence_after();
       // Stage dQ in the staging buffer, once the previous reductions have read it
-      // (the leader waits for them, then joins barrier 2).  K = 128: all boxes,
-      // then their reductions; K = 64: one 32-column box at a time.
+      // (the leader waits for them, then joins barrier 2).
       uint8_t* stage = smem + C::kDQS;
-      constexpr bool kOneBox = C::kDQSBoxes == 1;
-      auto reduce = [&](int b0, int nb) {
+      // K = 64: the one staged box (dims 32b .. 32b + 31) into the accumulator.
+      auto reduce_box = [&](int b) {
         fence_async_smem();
         named_sync(1, 128);
         if (leader) {
           BWD_TRACE(s, 17);
-          for (int b = b0; b < b0 + nb; ++b)
-            tma_reduce_add_4d(&tmDQ, stage + (kOneBox ? 0 : b * C::kDQSBox), 32 * b, h, q0 + m0,
-                              bidx);
+          tma_reduce_add_4d(&tmDQ, stage, 32 * b, h, q0 + m0, bidx);
           bulk_commit();
           bulk_wait_read();  // the staging buffer may be written again
         }
@@ -654,12 +661,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<float4*>(line + ((u ^ (row & 7)) << 4)) =
                 make_float4(__uint_as_float(v[4 * u]) * sc, __uint_as_float(v[4 * u + 1]) * sc,
                             __uint_as_float(v[4 * u + 2]) * sc, __uint_as_float(v[4 * u + 3]) * sc);
-          reduce(half, 1);
+          reduce_box(half);
         }
       } else {
+        // Half h (queries 32h .. 32h + 31) goes to buffer h; before a buffer is
+        // written again the leader has seen the reductions that read it two
+        // halves earlier complete (it keeps at most one group in flight).
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {  // 32 TMEM columns at a time
-          if (s > 0 && half == 0) named_sync(2, 128);
+          if (s > 0 || half > 0) named_sync(2, 128);
           uint32_t v[32];
           tmem_ld32(t_addr + 32 * half, v);
           tmem_ld_wait(v);
@@ -668,17 +678,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_warp(dq_empty);
           }
           // lane = dimension `row`, columns = queries 32 half .. +31: element
-          // (query q, dim row) of box row/32 at row q, byte 4 (row % 32), swizzled.
-          uint8_t* box = stage + (row >> 5) * C::kDQSBox;
+          // (query k, dim row) of box row/32 at row k, byte 4 (row % 32), swizzled.
+          uint8_t* buf = stage + half * (C::kDQSBoxes / 2) * C::kDQSBox;
+          uint8_t* box = buf + (row >> 5) * C::kDQSBox;
           const int piece = (row & 31) >> 2, word = (row & 3) * 4;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
             const int q = 32 * half + k;
             const float x = (m0 + q < q_len) ? __uint_as_float(v[k]) * a.scale : 0.f;
-            *reinterpret_cast<float*>(box + q * 128 + ((piece ^ (k & 7)) << 4) + word) = x;
+            *reinterpret_cast<float*>(box + k * 128 + ((piece ^ (k & 7)) << 4) + word) = x;
+          }
+          fence_async_smem();
+          named_sync(1, 128);
+          if (leader) {
+            BWD_TRACE(s, 17);
+#pragma unroll
+            for (int b = 0; b < D / 32; ++b)
+              tma_reduce_add_4d(&tmDQ, buf + b * C::kDQSBox, 32 * b, h, q0 + m0 + 32 * half, bidx);
+            bulk_commit();
+            bulk_wait_read_all_but_one();  // the other buffer may be written again
           }
         }
-        reduce(0, D / 32);
       }
     }
     if (leader) bulk_wait_all();
@@ -748,6 +768,10 @@ extern "C" int mea_bwd_trace_read(long long* host, int n) {
 #endif
 
 int bwd_query_block(int head_dim) { return head_dim == 128 ? BwdCfg<128>::BM : BwdCfg<64>::BM; }
+
+int bwd_dq_box_rows(int head_dim) {
+  return head_dim == 128 ? BwdCfg<128>::kDQRows : BwdCfg<64>::kDQRows;
+}
 
 cudaError_t launch_bwd(const BwdLaunch& L, cudaStream_t stream, int stages) {
   if (L.head_dim == 64)

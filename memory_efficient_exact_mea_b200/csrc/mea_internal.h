@@ -121,7 +121,7 @@ struct BwdArgs {
 
 struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // boxes: bwd_query_block rows (q, dout), kBwdBlock rows (k, v)
-  CUtensorMap tmDQ;                 // fp32 dq accumulator, 32 x 1 x bwd_query_block boxes
+  CUtensorMap tmDQ;                 // fp32 dq accumulator, 32 x 1 x bwd_dq_box_rows boxes
   BwdArgs args;
   int head_dim;
   bool bf16;
@@ -135,5 +135,6 @@ cudaError_t launch_bwd(const BwdLaunch& launch, cudaStream_t stream, int stages 
 
 // Query rows per step of the backward kernel for head dimension 64 or 128.
 int bwd_query_block(int head_dim);
+int bwd_dq_box_rows(int head_dim);  // rows of the dq accumulator's TMA reduction boxes
 
 }  // namespace mea
