@@ -76,9 +76,13 @@ def test_bwd_dense(mea, K, dtype, bias):
     _check(mea, p)
 
 
-@pytest.mark.parametrize("M,N", [(64, 64), (130, 70), (70, 130), (1, 5)])
-def test_bwd_rectangular_causal(mea, M, N):
-    p = synth.make_prefill(f"bwd_rect_{M}x{N}", 1, M, N, 2, 2, 64, "f16", "causal", seed=210 + M)
+@pytest.mark.parametrize("K,dtype", [(64, "f16"), (128, "bf16")])
+@pytest.mark.parametrize("M,N", [(64, 64), (130, 70), (70, 130), (1, 5), (97, 300)])
+def test_bwd_rectangular_causal(mea, M, N, K, dtype):
+    """Row counts that end inside a 32-query half step (K = 128 stages dQ per half)
+    and inside a 128-key block."""
+    p = synth.make_prefill(f"bwd_rect_{M}x{N}_{K}", 1, M, N, 2, 2, K, dtype, "causal",
+                           seed=210 + M)
     _check(mea, p)
 
 
