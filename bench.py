@@ -206,6 +206,7 @@ class ClockSampler:
         reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2])
                           if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_mhz_min": min(r[0] for r in loaded),
                 "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
                 "samples": len(rows), "samples_under_load": len(loaded)}
 
@@ -320,6 +321,9 @@ def run_ours(args, rank, world, local):
 
     # ---- the other workloads (secondary measurements) -----------------------
     also = {}
+    also_clk = ClockSampler(torch.cuda.current_device()) if not args.quick else None
+    if also_clk is not None:
+        also_clk.__enter__()
     if not args.quick:
         also["varlen_causal"] = measure_prefill(mea, synth.varlen_causal(), dev, stream, tc_peak)
         also["gqa_alibi_causal"] = measure_prefill(mea, synth.gqa_alibi_causal(), dev, stream,
@@ -334,6 +338,9 @@ def run_ours(args, rank, world, local):
                                                        stream, tc_peak)
         also["bwd_gqa_alibi_causal"] = measure_backward(mea, synth.gqa_alibi_causal(), dev,
                                                         stream, tc_peak)
+    if also_clk is not None:
+        also_clk.__exit__(None, None, None)
+        also["clocks"] = also_clk.summary()  # sampled over these secondary measurements
     assert mea.read_device_status() == 0
 
     traffic = traffic_for("fwd_sweep")
@@ -462,17 +469,23 @@ def measure_e2e(mea, sweep, dev, stream, args, world):
             "overlap": "uploads, kernels and downloads on three streams"}
 
 
-def _time(fn, stream, iters, warmup=3):
+def _time(fn, stream, iters, warmup=3, rounds=3):
+    """Mean time of one call over `iters` back-to-back calls, the best of `rounds`
+    such runs (a run that a clock dip or another tenant slowed is not the
+    kernel's time)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(iters):
-        fn()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / iters
+    best = float("inf")
+    for _ in range(rounds):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) / iters)
+    return best
 
 
 def measure_prefill(mea, p, dev, stream, tc_peak, iters=10, host_paths=False):
